@@ -1,0 +1,271 @@
+"""pkvq: attention over a paged, 8-bit-quantized KV cache on B200 (sm_100a).
+
+Thin Python binding of ``libpkvq.so`` (C ABI declared in include/pkvq.h).
+This module only marshals arguments: it checks tensor dtypes/devices/shapes,
+passes raw device pointers and the current CUDA stream, and turns status codes
+into exceptions.  Every step of the computation runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback, and loading fails loudly when
+the library has not been built.
+
+Entry points (same names as the C ABI, without the ``pkvq_`` prefix):
+  kv_write_quant, decode_workspace_bytes, paged_attn_decode,
+  paged_attn_prefill, device_status, status_string, version.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpkvq.so")
+LIB_CHECKED_PATH = os.path.join(_HERE, "libpkvq_checked.so")
+
+KV_FP8_E4M3 = 0
+KV_INT8 = 1
+
+EXPORTED = (
+    "pkvq_kv_write_quant",
+    "pkvq_decode_workspace_bytes",
+    "pkvq_paged_attn_decode",
+    "pkvq_paged_attn_prefill",
+    "pkvq_status_string",
+    "pkvq_device_status",
+    "pkvq_version",
+)
+
+
+class PkvqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class CacheStruct(ctypes.Structure):
+    _fields_ = [
+        ("dtype", ctypes.c_int32),
+        ("num_blocks", ctypes.c_int32),
+        ("block_size", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("k_cache", ctypes.c_void_p),
+        ("v_cache", ctypes.c_void_p),
+        ("k_scale", ctypes.c_void_p),
+        ("v_scale", ctypes.c_void_p),
+        ("k_scale_tok", ctypes.c_void_p),
+        ("v_scale_tok", ctypes.c_void_p),
+    ]
+
+
+_libs = {}
+
+
+def load_library(path: Optional[str] = None) -> ctypes.CDLL:
+    """Loads libpkvq.so (or another build of it); raises if it is missing."""
+    path = path or os.environ.get("PKVQ_LIBRARY", LIB_PATH)
+    if path in _libs:
+        return _libs[path]
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} not found: build the CUDA library first "
+            "(python -m paged_quantized_kv_quant_b200.build)")
+    lib = ctypes.CDLL(path)
+    P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    lib.pkvq_kv_write_quant.restype = I32
+    lib.pkvq_kv_write_quant.argtypes = [P, P, P, P, I32, P]
+    lib.pkvq_decode_workspace_bytes.restype = SZ
+    lib.pkvq_decode_workspace_bytes.argtypes = [I32, I32, I32, I32, P]
+    lib.pkvq_paged_attn_decode.restype = I32
+    lib.pkvq_paged_attn_decode.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, I32,
+                                           ctypes.c_float, P, SZ, P]
+    lib.pkvq_paged_attn_prefill.restype = I32
+    lib.pkvq_paged_attn_prefill.argtypes = [P, P, P, P, P, P, I32, P, I32, I32, I32,
+                                            ctypes.c_float, P, SZ, P]
+    lib.pkvq_status_string.restype = ctypes.c_char_p
+    lib.pkvq_status_string.argtypes = [I32]
+    lib.pkvq_device_status.restype = I32
+    lib.pkvq_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), I32]
+    lib.pkvq_version.restype = ctypes.c_char_p
+    lib.pkvq_version.argtypes = []
+    _libs[path] = lib
+    return lib
+
+
+def _lib():
+    return load_library()
+
+
+def status_string(status: int) -> str:
+    return _lib().pkvq_status_string(int(status)).decode()
+
+
+def version() -> str:
+    return _lib().pkvq_version().decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise PkvqError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+
+
+@dataclass
+class PagedKVCache:
+    """Caller-owned paged cache: codes [num_blocks][Hkv][block_size][D] uint8
+    (E4M3 bits or int8 two's complement), per-KV-head fp32 scales for FP8,
+    per-(block, head, token) fp16 scales for INT8."""
+    dtype: int
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    k_scale: Optional[torch.Tensor] = None
+    v_scale: Optional[torch.Tensor] = None
+    k_scale_tok: Optional[torch.Tensor] = None
+    v_scale_tok: Optional[torch.Tensor] = None
+
+    @staticmethod
+    def allocate(dtype: int, num_blocks: int, block_size: int, num_kv_heads: int,
+                 head_dim: int = 128, device="cuda", k_scale=None, v_scale=None):
+        shape = (num_blocks, num_kv_heads, block_size, head_dim)
+        kc = torch.zeros(shape, dtype=torch.uint8, device=device)
+        vc = torch.zeros(shape, dtype=torch.uint8, device=device)
+        if dtype == KV_FP8_E4M3:
+            ks = torch.as_tensor(k_scale, dtype=torch.float32).to(device).contiguous()
+            vs = torch.as_tensor(v_scale, dtype=torch.float32).to(device).contiguous()
+            return PagedKVCache(dtype, kc, vc, k_scale=ks, v_scale=vs)
+        kst = torch.zeros(shape[:3], dtype=torch.float16, device=device)
+        vst = torch.zeros(shape[:3], dtype=torch.float16, device=device)
+        return PagedKVCache(dtype, kc, vc, k_scale_tok=kst, v_scale_tok=vst)
+
+    @property
+    def num_blocks(self):
+        return self.k_cache.shape[0]
+
+    @property
+    def num_kv_heads(self):
+        return self.k_cache.shape[1]
+
+    @property
+    def block_size(self):
+        return self.k_cache.shape[2]
+
+    @property
+    def head_dim(self):
+        return self.k_cache.shape[3]
+
+    def struct(self) -> CacheStruct:
+        for name in ("k_cache", "v_cache"):
+            _need(getattr(self, name), torch.uint8, name, 4)
+        if self.dtype == KV_FP8_E4M3:
+            _need(self.k_scale, torch.float32, "k_scale", 1)
+            _need(self.v_scale, torch.float32, "v_scale", 1)
+        else:
+            _need(self.k_scale_tok, torch.float16, "k_scale_tok", 3)
+            _need(self.v_scale_tok, torch.float16, "v_scale_tok", 3)
+        nb, hkv, bs, d = self.k_cache.shape
+        return CacheStruct(self.dtype, nb, bs, hkv, d,
+                           self.k_cache.data_ptr(), self.v_cache.data_ptr(),
+                           self.k_scale.data_ptr() if self.k_scale is not None else None,
+                           self.v_scale.data_ptr() if self.v_scale is not None else None,
+                           self.k_scale_tok.data_ptr() if self.k_scale_tok is not None else None,
+                           self.v_scale_tok.data_ptr() if self.v_scale_tok is not None else None)
+
+
+def kv_write_quant(cache: PagedKVCache, k: torch.Tensor, v: torch.Tensor,
+                   slot_mapping: torch.Tensor, stream=None) -> None:
+    """Quantizes fp16 K/V [T][Hkv][D] into the cache slots (negative = skip)."""
+    _need(k, torch.float16, "k", 3)
+    _need(v, torch.float16, "v", 3)
+    _need(slot_mapping, torch.int32, "slot_mapping", 1)
+    cs = cache.struct()
+    _check(_lib().pkvq_kv_write_quant(ctypes.byref(cs), _ptr(k), _ptr(v), _ptr(slot_mapping),
+                                      int(slot_mapping.shape[0]), _stream(stream)),
+           "kv_write_quant")
+
+
+def decode_workspace_bytes(cache: PagedKVCache, batch: int, q_len: int, num_q_heads: int,
+                           max_context_len: int) -> int:
+    cs = cache.struct()
+    return int(_lib().pkvq_decode_workspace_bytes(batch, q_len, num_q_heads, max_context_len,
+                                                  ctypes.byref(cs)))
+
+
+def paged_attn_decode(cache: PagedKVCache, q: torch.Tensor, block_table: torch.Tensor,
+                      context_lens: torch.Tensor, max_context_len: int, softmax_scale: float,
+                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """q fp16 [B][q_len][Hq][D] -> out fp16 [B][q_len][Hq][D] (lse fp32 [B][q_len][Hq])."""
+    _need(q, torch.float16, "q", 4)
+    _need(block_table, torch.int32, "block_table", 2)
+    _need(context_lens, torch.int32, "context_lens", 1)
+    B, q_len, Hq, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, torch.float16, "out", 4)
+    if lse is not None:
+        _need(lse, torch.float32, "lse", 3)
+    need = decode_workspace_bytes(cache, B, q_len, Hq, max_context_len) if B else 0
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    cs = cache.struct()
+    _check(_lib().pkvq_paged_attn_decode(
+        ctypes.byref(cs), _ptr(q), _ptr(out), _ptr(lse), _ptr(block_table),
+        int(block_table.shape[1]), _ptr(context_lens), B, q_len, Hq, int(max_context_len),
+        float(softmax_scale), _ptr(workspace), wbytes, _stream(stream)), "paged_attn_decode")
+    return out
+
+
+def paged_attn_prefill(cache: PagedKVCache, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                       block_table: torch.Tensor, context_lens: torch.Tensor, max_q_len: int,
+                       softmax_scale: float, out: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """q fp16 [total_q][Hq][D] (packed varlen) -> out fp16 [total_q][Hq][D]."""
+    _need(q, torch.float16, "q", 3)
+    _need(cu_seqlens_q, torch.int32, "cu_seqlens_q", 1)
+    _need(block_table, torch.int32, "block_table", 2)
+    _need(context_lens, torch.int32, "context_lens", 1)
+    total_q, Hq, D = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, torch.float16, "out", 3)
+    if lse is not None:
+        _need(lse, torch.float32, "lse", 2)
+    B = int(context_lens.shape[0])
+    cs = cache.struct()
+    _check(_lib().pkvq_paged_attn_prefill(
+        ctypes.byref(cs), _ptr(q), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q), _ptr(block_table),
+        int(block_table.shape[1]), _ptr(context_lens), B, int(max_q_len), Hq,
+        float(softmax_scale), None, 0, _stream(stream)), "paged_attn_prefill")
+    return out
+
+
+def device_status(clear: bool = True) -> int:
+    """Device status word (0 = no device-side check fired); synchronizes."""
+    v = ctypes.c_uint32(0)
+    _check(_lib().pkvq_device_status(ctypes.byref(v), 1 if clear else 0), "device_status")
+    return int(v.value)

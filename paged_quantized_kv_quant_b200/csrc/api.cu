@@ -1,0 +1,359 @@
+// C ABI of libpkvq.so: argument validation, tensor-map setup and dispatch.
+// Every check happens on the host before any launch; nothing here allocates
+// device memory or synchronizes the host with the device (except
+// pkvq_device_status, a diagnostic).
+#include "../../include/pkvq.h"
+#include "common.cuh"
+#include "internal.h"
+
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <mutex>
+#include <stdlib.h>
+
+namespace pkvq {
+
+__device__ uint32_t g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+uint32_t *status_ptr()
+{
+    static uint32_t *ptrs[kMaxDevices] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess)
+            return nullptr;
+        ptrs[dev] = static_cast<uint32_t *>(p);
+    }
+    return ptrs[dev];
+}
+
+bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+pkvq_status check_cache(const pkvq_cache *c)
+{
+    if (!c || !c->k_cache || !c->v_cache)
+        return PKVQ_ERR_INVALID_ARG;
+    if (c->dtype != PKVQ_KV_FP8_E4M3 && c->dtype != PKVQ_KV_INT8)
+        return PKVQ_ERR_UNSUPPORTED;
+    if (c->head_dim != kHeadDim)
+        return PKVQ_ERR_UNSUPPORTED;
+    if (c->block_size != 16 && c->block_size != 32 && c->block_size != 64)
+        return PKVQ_ERR_UNSUPPORTED;
+    if (c->num_blocks <= 0 || c->num_kv_heads <= 0)
+        return PKVQ_ERR_INVALID_ARG;
+    // tensor-map row coordinates are int32
+    if ((long long)c->num_blocks * c->num_kv_heads * c->block_size >= (1LL << 31))
+        return PKVQ_ERR_UNSUPPORTED;
+    if (c->dtype == PKVQ_KV_FP8_E4M3) {
+        if (!c->k_scale || !c->v_scale)
+            return PKVQ_ERR_INVALID_ARG;
+    } else {
+        if (!c->k_scale_tok || !c->v_scale_tok)
+            return PKVQ_ERR_INVALID_ARG;
+        if (!aligned16(c->k_scale_tok) || !aligned16(c->v_scale_tok))
+            return PKVQ_ERR_MISALIGNED;
+    }
+    if (!aligned16(c->k_cache) || !aligned16(c->v_cache))
+        return PKVQ_ERR_MISALIGNED;
+    return PKVQ_OK;
+}
+
+pkvq_status cache_maps(const pkvq_cache *c, CUtensorMap *km, CUtensorMap *vm)
+{
+    const uint64_t rows = (uint64_t)c->num_blocks * c->num_kv_heads * c->block_size;
+    if (!make_cache_tensor_map(km, c->k_cache, rows, c->block_size) ||
+        !make_cache_tensor_map(vm, c->v_cache, rows, c->block_size))
+        return PKVQ_ERR_CUDA;
+    return PKVQ_OK;
+}
+
+pkvq_status from_cuda(cudaError_t e)
+{
+    return e == cudaSuccess ? PKVQ_OK : PKVQ_ERR_CUDA;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace
+
+bool make_cache_tensor_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[2] = {128, rows};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int device_sm_count()
+{
+    static int counts[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return 148;
+    if (!counts[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        counts[dev] = n;
+    }
+    return counts[dev];
+}
+
+}  // namespace pkvq
+
+using namespace pkvq;
+
+extern "C" {
+
+const char *pkvq_version(void)
+{
+    return "0.1.0";
+}
+
+const char *pkvq_status_string(pkvq_status s)
+{
+    switch (s) {
+    case PKVQ_OK: return "ok";
+    case PKVQ_ERR_INVALID_ARG: return "invalid argument";
+    case PKVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PKVQ_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case PKVQ_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case PKVQ_ERR_DEVICE: return "device-side check failed";
+    case PKVQ_ERR_CUDA: return "CUDA runtime error";
+    }
+    return "unknown status";
+}
+
+pkvq_status pkvq_device_status(uint32_t *status_out, int32_t clear)
+{
+    if (!status_out)
+        return PKVQ_ERR_INVALID_ARG;
+    uint32_t *p = status_ptr();
+    if (!p)
+        return PKVQ_ERR_CUDA;
+    if (cudaMemcpy(status_out, p, sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return PKVQ_ERR_CUDA;
+    if (clear && cudaMemset(p, 0, sizeof(uint32_t)) != cudaSuccess)
+        return PKVQ_ERR_CUDA;
+    return PKVQ_OK;
+}
+
+pkvq_status pkvq_kv_write_quant(const pkvq_cache *cache, const void *k, const void *v,
+                                const int32_t *slot_mapping, int32_t num_tokens, void *stream)
+{
+    pkvq_status st = check_cache(cache);
+    if (st != PKVQ_OK)
+        return st;
+    if (num_tokens < 0)
+        return PKVQ_ERR_INVALID_ARG;
+    if (num_tokens == 0)
+        return PKVQ_OK;
+    if (!k || !v || !slot_mapping)
+        return PKVQ_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v))
+        return PKVQ_ERR_MISALIGNED;
+    KvWriteParams p{};
+    p.k_cache = static_cast<uint8_t *>(cache->k_cache);
+    p.v_cache = static_cast<uint8_t *>(cache->v_cache);
+    p.k_scale = cache->k_scale;
+    p.v_scale = cache->v_scale;
+    p.k_scale_tok = static_cast<uint16_t *>(cache->k_scale_tok);
+    p.v_scale_tok = static_cast<uint16_t *>(cache->v_scale_tok);
+    p.k = static_cast<const __half *>(k);
+    p.v = static_cast<const __half *>(v);
+    p.slot_mapping = slot_mapping;
+    p.num_tokens = num_tokens;
+    p.num_kv_heads = cache->num_kv_heads;
+    p.num_blocks = cache->num_blocks;
+    p.block_size = cache->block_size;
+    p.status = status_ptr();
+    if (!p.status)
+        return PKVQ_ERR_CUDA;
+    return from_cuda(launch_kv_write_quant(p, cache->dtype, static_cast<cudaStream_t>(stream)));
+}
+
+size_t pkvq_decode_workspace_bytes(int32_t batch, int32_t q_len, int32_t num_q_heads,
+                                   int32_t max_context_len, const pkvq_cache *cache)
+{
+    if (check_cache(cache) != PKVQ_OK || batch <= 0 || q_len <= 0 || q_len > 16 ||
+        max_context_len < 0 || num_q_heads <= 0 || num_q_heads % cache->num_kv_heads)
+        return 0;
+    DecodePlan plan;
+    if (!decode_plan(batch, q_len, num_q_heads, cache->num_kv_heads, cache->block_size,
+                     max_context_len, &plan))
+        return 0;
+    return plan.workspace_bytes;
+}
+
+pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void *q, void *out,
+                                   float *lse_out, const int32_t *block_table,
+                                   int32_t max_blocks_per_seq, const int32_t *context_lens,
+                                   int32_t batch, int32_t q_len, int32_t num_q_heads,
+                                   int32_t max_context_len, float softmax_scale,
+                                   void *workspace, size_t workspace_bytes, void *stream)
+{
+    pkvq_status st = check_cache(cache);
+    if (st != PKVQ_OK)
+        return st;
+    if (batch < 0 || q_len < 1 || q_len > 16 || num_q_heads <= 0 || max_context_len < 0 ||
+        max_blocks_per_seq < 0)
+        return PKVQ_ERR_INVALID_ARG;
+    if (num_q_heads % cache->num_kv_heads)
+        return PKVQ_ERR_INVALID_ARG;
+    const int group = num_q_heads / cache->num_kv_heads;
+    if (group > 16)
+        return PKVQ_ERR_UNSUPPORTED;
+    if (!isfinite(softmax_scale))
+        return PKVQ_ERR_INVALID_ARG;
+    if (batch == 0)
+        return PKVQ_OK;
+    if (!q || !out || !block_table || !context_lens)
+        return PKVQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out))
+        return PKVQ_ERR_MISALIGNED;
+    if ((long long)max_blocks_per_seq * cache->block_size < max_context_len)
+        return PKVQ_ERR_INVALID_ARG;
+    DecodePlan plan;
+    if (!decode_plan(batch, q_len, num_q_heads, cache->num_kv_heads, cache->block_size,
+                     max_context_len, &plan))
+        return PKVQ_ERR_INVALID_ARG;
+    if (plan.workspace_bytes > 0) {
+        if (!workspace || workspace_bytes < plan.workspace_bytes)
+            return PKVQ_ERR_WORKSPACE_TOO_SMALL;
+        if (!aligned16(workspace))
+            return PKVQ_ERR_MISALIGNED;
+    }
+    CUtensorMap km, vm;
+    st = cache_maps(cache, &km, &vm);
+    if (st != PKVQ_OK)
+        return st;
+    DecodeParams p{};
+    p.k_scale = cache->k_scale;
+    p.v_scale = cache->dtype == PKVQ_KV_FP8_E4M3 ? cache->v_scale : nullptr;
+    p.k_scale_tok = static_cast<const uint16_t *>(cache->k_scale_tok);
+    p.v_scale_tok = static_cast<const uint16_t *>(cache->v_scale_tok);
+    p.q = static_cast<const __half *>(q);
+    p.out = static_cast<__half *>(out);
+    p.lse = lse_out;
+    p.block_table = block_table;
+    p.context_lens = context_lens;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.batch = batch;
+    p.q_len = q_len;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = cache->num_kv_heads;
+    p.group = group;
+    p.num_blocks = cache->num_blocks;
+    p.block_size = cache->block_size;
+    p.rows = q_len * group;
+    p.rows_per_cta = plan.rows_per_cta;
+    p.row_groups = plan.row_groups;
+    p.num_splits = plan.num_splits;
+    p.blocks_per_split = plan.blocks_per_split;
+    p.scale_log2 = softmax_scale * kLog2e;
+    float *ws = static_cast<float *>(workspace);
+    const size_t n_rows_ws =
+        (size_t)batch * cache->num_kv_heads * plan.num_splits * p.rows;
+    p.ws_o = plan.workspace_bytes ? ws : nullptr;
+    p.ws_ml = plan.workspace_bytes ? ws + n_rows_ws * kHeadDim : nullptr;
+    p.status = status_ptr();
+    if (!p.status)
+        return PKVQ_ERR_CUDA;
+    return from_cuda(launch_decode(p, plan, cache->dtype, km, vm, static_cast<cudaStream_t>(stream)));
+}
+
+pkvq_status pkvq_paged_attn_prefill(const pkvq_cache *cache, const void *q, void *out,
+                                    float *lse_out, const int32_t *cu_seqlens_q,
+                                    const int32_t *block_table, int32_t max_blocks_per_seq,
+                                    const int32_t *context_lens, int32_t batch,
+                                    int32_t max_q_len, int32_t num_q_heads,
+                                    float softmax_scale, void *workspace,
+                                    size_t workspace_bytes, void *stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    pkvq_status st = check_cache(cache);
+    if (st != PKVQ_OK)
+        return st;
+    if (batch < 0 || max_q_len < 0 || num_q_heads <= 0 || max_blocks_per_seq < 0)
+        return PKVQ_ERR_INVALID_ARG;
+    if (num_q_heads % cache->num_kv_heads)
+        return PKVQ_ERR_INVALID_ARG;
+    const int group = num_q_heads / cache->num_kv_heads;
+    if (group > 128)
+        return PKVQ_ERR_UNSUPPORTED;
+    if (!isfinite(softmax_scale))
+        return PKVQ_ERR_INVALID_ARG;
+    if (batch == 0 || max_q_len == 0)
+        return PKVQ_OK;
+    if (!q || !out || !cu_seqlens_q || !block_table || !context_lens)
+        return PKVQ_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out))
+        return PKVQ_ERR_MISALIGNED;
+    CUtensorMap km, vm;
+    st = cache_maps(cache, &km, &vm);
+    if (st != PKVQ_OK)
+        return st;
+    PrefillParams p{};
+    p.k_scale = cache->k_scale;
+    p.v_scale = cache->v_scale;
+    p.k_scale_tok = static_cast<const uint16_t *>(cache->k_scale_tok);
+    p.v_scale_tok = static_cast<const uint16_t *>(cache->v_scale_tok);
+    p.q = static_cast<const __half *>(q);
+    p.out = static_cast<__half *>(out);
+    p.lse = lse_out;
+    p.cu_seqlens_q = cu_seqlens_q;
+    p.block_table = block_table;
+    p.context_lens = context_lens;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.batch = batch;
+    p.max_q_len = max_q_len;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = cache->num_kv_heads;
+    p.group = group;
+    p.num_blocks = cache->num_blocks;
+    p.block_size = cache->block_size;
+    p.tokens_per_tile = 128 / group;
+    p.q_tiles = (max_q_len + p.tokens_per_tile - 1) / p.tokens_per_tile;
+    p.scale_log2 = softmax_scale * kLog2e;
+    p.status = status_ptr();
+    if (!p.status)
+        return PKVQ_ERR_CUDA;
+    return from_cuda(launch_prefill(p, cache->dtype, km, vm, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

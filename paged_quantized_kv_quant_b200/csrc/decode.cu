@@ -1,0 +1,599 @@
+// Split-KV decode / draft-verify attention over the paged 8-bit cache.
+//
+// Source: "1Cat-LLM" README, "Layer 1" (paged KV is read through page ids
+// with wide aligned loads, the page id reused for a whole page), "Layer 2"
+// (GQA multi-head packing into wider tensor-core work, online softmax with
+// FP32 state, Split-KV with an FP32 merge of the partial states) and
+// "128-bit Loads" (fewer, wider, aligned cache loads).
+//
+// Work decomposition.  A CTA owns one (sequence, KV head, row group, split):
+// the rows are the q_len x G query rows that share the KV head (GQA packing),
+// the split is a contiguous range of cache blocks.  Each of its 4 warps
+// streams whole cache blocks (block_size x 128 codes of K and of V, one
+// contiguous tile each) through a private ring of TMA stages: lane 0 issues a
+// 2-D tensor copy per tile with 128-byte swizzle, so the fragment loads below
+// are free of shared-memory bank conflicts.
+//
+// Tensor-core mapping (legacy mma.sync m16n8k16, fp16 x fp16 -> fp32).  The
+// contraction puts KEYS on M and query ROWS on N: S^T = K Q^T and
+// O^T += V^T P^T.  With G = 8 a decode step's rows fill one n8 tile exactly,
+// so no tensor-core work is padded.  Codes are converted to fp16 in registers
+// straight into A fragments (E4M3 and int8 values are exact in fp16); the head
+// dimension is permuted consistently between Q and K so that every thread
+// reads 32 contiguous code bytes per key.  P^T reaches the B-operand layout
+// through movmatrix.trans, without shared memory.
+//
+// Scales.  FP8: the per-head K scale folds into the score multiplier and the
+// per-head V scale into the final normalisation.  INT8: the per-token K scale
+// multiplies score columns in fp32; the per-token V scale multiplies the
+// dequantised V in fp16 before the PV product (P itself stays unscaled, so
+// small probabilities never meet small scales in fp16).
+#include "common.cuh"
+#include "internal.h"
+
+#include <math.h>
+
+namespace pkvq {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr float kLn2 = 0.693147180559945309f;
+
+template <int BS>
+struct DecodeCfg {
+    static constexpr int kStages = BS == 16 ? 4 : (BS == 32 ? 3 : 2);
+    static constexpr int kTileBytes = BS * 128;
+    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kScaleHalves = 2 * BS;     // K then V scales of one block
+    static constexpr int kMT = BS / 16;             // 16-key m-tiles per block
+};
+
+template <int BS>
+constexpr size_t decode_smem_bytes()
+{
+    using C = DecodeCfg<BS>;
+    return 1024 + (size_t)kWarps * C::kStages * C::kStageBytes +
+           (size_t)kWarps * C::kStages * C::kScaleHalves * 2 + (size_t)kWarps * C::kStages * 8;
+}
+
+__device__ __forceinline__ uint4 lds128(const uint8_t *p)
+{
+    return *reinterpret_cast<const uint4 *>(p);
+}
+
+template <int KVT>
+__device__ __forceinline__ uint32_t cvt2(uint32_t pair)
+{
+    if constexpr (KVT == kKvFp8)
+        return e4m3x2_to_half2(pair);
+    else
+        return s8x2_to_half2(pair);
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b)
+{
+    __half2 r = __hmul2(*reinterpret_cast<__half2 *>(&a), *reinterpret_cast<__half2 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
+{
+    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+template <int KVT, int NT, int BS>
+__global__ void __launch_bounds__(kThreads)
+decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
+                    const __grid_constant__ CUtensorMap vmap, const DecodeParams p)
+{
+    using C = DecodeCfg<BS>;
+    constexpr int S = C::kStages;
+    constexpr int RC = 8 * NT;
+    constexpr int MT = C::kMT;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *tiles = smem;
+    uint16_t *scales = reinterpret_cast<uint16_t *>(tiles + kWarps * S * C::kStageBytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(scales + kWarps * S * C::kScaleHalves);
+
+    const int split = blockIdx.x;
+    const int h = blockIdx.y % p.num_kv_heads;
+    const int rg = blockIdx.y / p.num_kv_heads;
+    const int b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+
+    // Let the merge kernel (programmatic dependent launch) get scheduled early;
+    // it still waits for this grid to finish before reading the workspace.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    if (device_wait_failed(p.status))
+        return;
+    const int ctx = p.context_lens[b];
+    const int nblk_seq = (ctx + BS - 1) / BS;
+    const int blk_begin = split * p.blocks_per_split;
+    if (p.num_splits > 1 && blk_begin >= nblk_seq)
+        return;   // the merge kernel only reads splits that hold keys
+    const int nblk = max(0, min(nblk_seq, blk_begin + p.blocks_per_split) - blk_begin);
+    const int n_it = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
+
+    uint64_t *my_bars = bars + warp * S;
+    uint8_t *my_tiles = tiles + warp * S * C::kStageBytes;
+    uint16_t *my_scales = scales + warp * S * C::kScaleHalves;
+    if (lane == 0) {
+        prefetch_tmap(&kmap);
+        prefetch_tmap(&vmap);
+#pragma unroll
+        for (int s = 0; s < S; ++s)
+            mbar_init(&my_bars[s], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    // ---- query fragments (B operand of S^T = K Q^T), loop invariant ----
+    const int h0 = h * p.group;
+    uint32_t qf[NT][8][2];
+    int pos[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int r = rg * RC + nt * 8 + g;
+        uint32_t u[16];
+        if (r < p.rows) {
+            const int tq = r / p.group, gq = r % p.group;
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                p.q + (((size_t)b * p.q_len + tq) * p.num_q_heads + h0 + gq) * kHeadDim + 32 * t);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint4 w = __ldg(src + i);
+                u[4 * i] = w.x, u[4 * i + 1] = w.y, u[4 * i + 2] = w.z, u[4 * i + 3] = w.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                u[i] = 0u;
+        }
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            qf[nt][ks][0] = u[2 * ks];       // d = 32t + 4ks + {0,1}
+            qf[nt][ks][1] = u[2 * ks + 1];   // d = 32t + 4ks + {2,3}
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int rr = rg * RC + nt * 8 + 2 * t + i;
+            pos[nt][i] = rr < p.rows ? ctx - p.q_len + rr / p.group : ctx - 1;
+        }
+    }
+
+    float kfac = p.scale_log2;
+    if constexpr (KVT == kKvFp8)
+        kfac *= __ldg(p.k_scale + h);
+
+    float o[NT][8][4];
+    float m[NT][2], l[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int dt = 0; dt < 8; ++dt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                o[nt][dt][c] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+            m[nt][i] = -INFINITY, l[nt][i] = 0.0f;
+    }
+
+    // ---- block ids: a sliding window of 64 iterations held in two registers ----
+    const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq;
+    auto lblk = [&](int it) { return blk_begin + warp + kWarps * it; };
+    int win0 = lane < n_it ? __ldg(bt + lblk(lane)) : 0;
+    int win1 = 32 + lane < n_it ? __ldg(bt + lblk(32 + lane)) : 0;
+    int win_base = 0;
+
+    constexpr uint32_t kTx = C::kStageBytes + (KVT == kKvInt8 ? C::kScaleHalves * 2 : 0);
+    auto issue = [&](int j) {   // warp-uniform call
+        const int a = __shfl_sync(0xffffffffu, win0, j & 31);
+        const int c = __shfl_sync(0xffffffffu, win1, j & 31);
+        int phys = (j - win_base) < 32 ? a : c;
+        if (lane == 0) {
+#ifdef PKVQ_BOUNDS_CHECK
+            if (phys < 0 || phys >= p.num_blocks) {
+                atomicOr(p.status, kStatusBadBlock);
+                phys = 0;
+            }
+#endif
+            const int stage = j % S;
+            uint64_t *bar = &my_bars[stage];
+            mbar_arrive_expect_tx(bar, kTx);
+            const int y = (phys * p.num_kv_heads + h) * BS;
+            uint8_t *dst = my_tiles + stage * C::kStageBytes;
+            tma_tile_2d_g2s(dst, &kmap, 0, y, bar);
+            tma_tile_2d_g2s(dst + C::kTileBytes, &vmap, 0, y, bar);
+            if constexpr (KVT == kKvInt8) {
+                uint16_t *sd = my_scales + stage * C::kScaleHalves;
+                tma_bulk_g2s(sd, p.k_scale_tok + (size_t)y, BS * 2, bar);
+                tma_bulk_g2s(sd + BS, p.v_scale_tok + (size_t)y, BS * 2, bar);
+            }
+        }
+    };
+
+    int issued = 0;
+    for (; issued < S && issued < n_it; ++issued)
+        issue(issued);
+
+    const int min_pos = ctx - p.q_len;
+    int it = 0;
+    bool ok = true;
+    for (; it < n_it; ++it) {
+        const int stage = it % S;
+        if (!mbar_wait(&my_bars[stage], (it / S) & 1, p.status)) {
+            ok = false;
+            break;
+        }
+        const uint8_t *kt = my_tiles + stage * C::kStageBytes;
+        const uint8_t *vt = kt + C::kTileBytes;
+        const uint16_t *st = my_scales + stage * C::kScaleHalves;
+        const int key0 = lblk(it) * BS;
+
+        // ---------------- S^T = K Q^T ----------------
+        float sc[MT][NT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int r0 = mt * 16 + g;   // key rows r0 and r0 + 8; (row & 7) == g
+            const uint4 ka0 = lds128(kt + r0 * 128 + (((2 * t) ^ g) << 4));
+            const uint4 ka1 = lds128(kt + r0 * 128 + (((2 * t + 1) ^ g) << 4));
+            const uint4 kb0 = lds128(kt + (r0 + 8) * 128 + (((2 * t) ^ g) << 4));
+            const uint4 kb1 = lds128(kt + (r0 + 8) * 128 + (((2 * t + 1) ^ g) << 4));
+            const uint32_t wa[8] = {ka0.x, ka0.y, ka0.z, ka0.w, ka1.x, ka1.y, ka1.z, ka1.w};
+            const uint32_t wb[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    sc[mt][nt][c] = 0.0f;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t a[4] = {cvt2<KVT>(wa[ks] & 0xffffu), cvt2<KVT>(wb[ks] & 0xffffu),
+                                       cvt2<KVT>(wa[ks] >> 16), cvt2<KVT>(wb[ks] >> 16)};
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    mma_f16_16816(sc[mt][nt], a, qf[nt][ks]);
+            }
+            float f0 = kfac, f1 = kfac;
+            if constexpr (KVT == kKvInt8) {
+                f0 *= __half2float(__ushort_as_half(st[r0]));
+                f1 *= __half2float(__ushort_as_half(st[r0 + 8]));
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                sc[mt][nt][0] *= f0, sc[mt][nt][1] *= f0;
+                sc[mt][nt][2] *= f1, sc[mt][nt][3] *= f1;
+            }
+        }
+
+        // causal / context mask, only where a key can lie past a row's position
+        if (key0 + BS - 1 > min_pos) {
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int key = key0 + mt * 16 + g + (c >> 1) * 8;
+                        if (key > pos[nt][c & 1])
+                            sc[mt][nt][c] = -INFINITY;
+                    }
+        }
+
+        // ---------------- online softmax (base 2) ----------------
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+                    mx = fmaxf(mx, fmaxf(sc[mt][nt][i], sc[mt][nt][2 + i]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                const float m_new = fmaxf(m[nt][i], mx);
+                const float m_use = m_new == -INFINITY ? 0.0f : m_new;
+                const float corr = fast_exp2(m[nt][i] - m_use);
+                m[nt][i] = m_new;
+                float ls = l[nt][i] * corr;
+#pragma unroll
+                for (int dt = 0; dt < 8; ++dt) {
+                    o[nt][dt][i] *= corr;
+                    o[nt][dt][2 + i] *= corr;
+                }
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    const float p0 = fast_exp2(sc[mt][nt][i] - m_use);
+                    const float p1 = fast_exp2(sc[mt][nt][2 + i] - m_use);
+                    sc[mt][nt][i] = p0;
+                    sc[mt][nt][2 + i] = p1;
+                    ls += p0 + p1;
+                }
+                l[nt][i] = ls;
+            }
+        }
+
+        // ---------------- O^T += V^T P^T ----------------
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            uint32_t pb[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                pb[nt][0] = movmatrix_trans(pack_half2(sc[mt][nt][0], sc[mt][nt][1]));
+                pb[nt][1] = movmatrix_trans(pack_half2(sc[mt][nt][2], sc[mt][nt][3]));
+            }
+            const int r0 = mt * 16 + 2 * t;   // key rows r0, r0+1, r0+8, r0+9
+            uint4 v0 = lds128(vt + r0 * 128 + ((g ^ (r0 & 7)) << 4));
+            uint4 v1 = lds128(vt + (r0 + 1) * 128 + ((g ^ ((r0 + 1) & 7)) << 4));
+            uint4 v2 = lds128(vt + (r0 + 8) * 128 + ((g ^ ((r0 + 8) & 7)) << 4));
+            uint4 v3 = lds128(vt + (r0 + 9) * 128 + ((g ^ ((r0 + 9) & 7)) << 4));
+            uint32_t s01 = 0u, s23 = 0u;
+            if constexpr (KVT == kKvInt8) {
+                s01 = (uint32_t)st[BS + r0] | ((uint32_t)st[BS + r0 + 1] << 16);
+                s23 = (uint32_t)st[BS + r0 + 8] | ((uint32_t)st[BS + r0 + 9] << 16);
+            }
+            if (key0 + BS > ctx) {
+                // Slots past the context were never written: their codes (and
+                // INT8 scales) may be NaN patterns, and 0 * NaN would poison O.
+                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                const int k0 = key0 + r0;
+                if (k0 >= ctx) v0 = z, s01 &= 0xffff0000u;
+                if (k0 + 1 >= ctx) v1 = z, s01 &= 0x0000ffffu;
+                if (k0 + 8 >= ctx) v2 = z, s23 &= 0xffff0000u;
+                if (k0 + 9 >= ctx) v3 = z, s23 &= 0x0000ffffu;
+            }
+#pragma unroll
+            for (int dt = 0; dt < 8; ++dt) {
+                const int wi = dt >> 1;
+                const uint32_t bo = 2u * (dt & 1);
+                const uint32_t x0 = word_of(v0, wi), x1 = word_of(v1, wi);
+                const uint32_t x2 = word_of(v2, wi), x3 = word_of(v3, wi);
+                const uint32_t sel0 = bo | ((4u + bo) << 4);
+                const uint32_t sel1 = (bo + 1u) | ((5u + bo) << 4);
+                uint32_t a[4] = {cvt2<KVT>(__byte_perm(x0, x1, sel0) & 0xffffu),
+                                 cvt2<KVT>(__byte_perm(x0, x1, sel1) & 0xffffu),
+                                 cvt2<KVT>(__byte_perm(x2, x3, sel0) & 0xffffu),
+                                 cvt2<KVT>(__byte_perm(x2, x3, sel1) & 0xffffu)};
+                if constexpr (KVT == kKvInt8) {
+                    a[0] = hmul2_u32(a[0], s01);
+                    a[1] = hmul2_u32(a[1], s01);
+                    a[2] = hmul2_u32(a[2], s23);
+                    a[3] = hmul2_u32(a[3], s23);
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    mma_f16_16816(o[nt][dt], a, pb[nt]);
+            }
+        }
+
+        __syncwarp();
+        if (issued < n_it) {
+            issue(issued);
+            ++issued;
+        }
+        if ((it & 31) == 31) {
+            win_base += 32;
+            win0 = win1;
+            win1 = win_base + 32 + lane < n_it ? __ldg(bt + lblk(win_base + 32 + lane)) : 0;
+        }
+    }
+    if (!ok) {
+        // A wait gave up: let the copies still in flight land (bounded) before
+        // this CTA's shared memory is reused or released.
+        for (int j = it; j < issued; ++j)
+            mbar_wait(&my_bars[j % S], (j / S) & 1, nullptr);
+    }
+
+    // row sums: reduce the per-thread partial sums over the 8 key lanes
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            float s = l[nt][i];
+            s += __shfl_xor_sync(0xffffffffu, s, 4);
+            s += __shfl_xor_sync(0xffffffffu, s, 8);
+            s += __shfl_xor_sync(0xffffffffu, s, 16);
+            l[nt][i] = s;
+        }
+
+    // ---- merge the 4 warps' states through shared memory (tiles are idle now) ----
+    __syncthreads();
+    float *so = reinterpret_cast<float *>(smem);      // [W][RC][128]
+    float *sm = so + kWarps * RC * kHeadDim;          // [W][RC]
+    float *sl = sm + kWarps * RC;                     // [W][RC]
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int r = nt * 8 + 2 * t + i;
+            float *dst = so + (warp * RC + r) * kHeadDim + 16 * g;
+#pragma unroll
+            for (int dt = 0; dt < 8; ++dt) {
+                dst[2 * dt] = o[nt][dt][i];
+                dst[2 * dt + 1] = o[nt][dt][2 + i];
+            }
+            if (g == 0) {
+                sm[warp * RC + r] = m[nt][i];
+                sl[warp * RC + r] = l[nt][i];
+            }
+        }
+    __syncthreads();
+
+    const int d = threadIdx.x;   // 128 threads <-> 128 dims
+    float vfac = 1.0f;
+    if constexpr (KVT == kKvFp8)
+        vfac = __ldg(p.v_scale + h);
+    for (int r = 0; r < RC; ++r) {
+        const int rr = rg * RC + r;
+        if (rr >= p.rows)
+            break;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+            M = fmaxf(M, sm[w * RC + r]);
+        const float Mu = M == -INFINITY ? 0.0f : M;
+        float L = 0.0f, O = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const float e = fast_exp2(sm[w * RC + r] - Mu);
+            L += sl[w * RC + r] * e;
+            O += so[(w * RC + r) * kHeadDim + d] * e;
+        }
+        if (p.num_splits == 1) {
+            const int tq = rr / p.group, gq = rr % p.group;
+            const size_t orow = ((size_t)b * p.q_len + tq) * p.num_q_heads + h0 + gq;
+            p.out[orow * kHeadDim + d] = __float2half_rn(L > 0.0f ? O / L * vfac : 0.0f);
+            if (d == 0 && p.lse)
+                p.lse[orow] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        } else {
+            const size_t wrow =
+                (((size_t)b * p.num_kv_heads + h) * p.num_splits + split) * p.rows + rr;
+            p.ws_o[wrow * kHeadDim + d] = O;
+            if (d == 0) {
+                p.ws_ml[wrow * 2] = M;
+                p.ws_ml[wrow * 2 + 1] = L;
+            }
+        }
+    }
+}
+
+// Merge of the split partial states (one warp per output row):
+// M = max_i m_i, L = sum_i l_i 2^(m_i - M), O = sum_i O_i 2^(m_i - M) / L.
+__global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long gw = (long long)blockIdx.x * 4 + warp;
+    const long long total = (long long)p.batch * p.num_kv_heads * p.rows;
+    if (gw >= total)
+        return;
+    const int rr = (int)(gw % p.rows);
+    const int h = (int)((gw / p.rows) % p.num_kv_heads);
+    const int b = (int)(gw / ((long long)p.rows * p.num_kv_heads));
+    const int ctx = p.context_lens[b];
+    const int nblk = (ctx + p.block_size - 1) / p.block_size;
+    const int nvalid = min(p.num_splits, (nblk + p.blocks_per_split - 1) / p.blocks_per_split);
+    const size_t base = ((size_t)b * p.num_kv_heads + h) * p.num_splits * p.rows + rr;
+    float M = -INFINITY;
+    for (int s = 0; s < nvalid; ++s)
+        M = fmaxf(M, p.ws_ml[(base + (size_t)s * p.rows) * 2]);
+    const float Mu = M == -INFINITY ? 0.0f : M;
+    float L = 0.0f;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < nvalid; ++s) {
+        const size_t wrow = base + (size_t)s * p.rows;
+        const float e = fast_exp2(p.ws_ml[wrow * 2] - Mu);
+        L += p.ws_ml[wrow * 2 + 1] * e;
+        const float4 v = reinterpret_cast<const float4 *>(p.ws_o + wrow * kHeadDim)[lane];
+        O.x += v.x * e, O.y += v.y * e, O.z += v.z * e, O.w += v.w * e;
+    }
+    const float vfac = p.v_scale ? __ldg(p.v_scale + h) : 1.0f;
+    const int tq = rr / p.group, gq = rr % p.group;
+    const size_t orow = ((size_t)b * p.q_len + tq) * p.num_q_heads + h * p.group + gq;
+    __half2 lo = __floats2half2_rn(L > 0.0f ? O.x / L * vfac : 0.0f, L > 0.0f ? O.y / L * vfac : 0.0f);
+    __half2 hi = __floats2half2_rn(L > 0.0f ? O.z / L * vfac : 0.0f, L > 0.0f ? O.w / L * vfac : 0.0f);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t *>(&lo);
+    pk.y = *reinterpret_cast<uint32_t *>(&hi);
+    reinterpret_cast<uint2 *>(p.out + orow * kHeadDim)[lane] = pk;
+    if (lane == 0 && p.lse)
+        p.lse[orow] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
+}
+
+template <int KVT, int NT, int BS>
+cudaError_t launch_split(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                         cudaStream_t stream)
+{
+    constexpr size_t smem = decode_smem_bytes<BS>();
+    auto kern = decode_split_kernel<KVT, NT, BS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    dim3 grid(p.num_splits, p.num_kv_heads * p.row_groups, p.batch);
+    kern<<<grid, kThreads, smem, stream>>>(kmap, vmap, p);
+    return cudaGetLastError();
+}
+
+template <int KVT, int NT>
+cudaError_t launch_bs(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                      cudaStream_t stream)
+{
+    switch (p.block_size) {
+    case 16: return launch_split<KVT, NT, 16>(p, kmap, vmap, stream);
+    case 32: return launch_split<KVT, NT, 32>(p, kmap, vmap, stream);
+    case 64: return launch_split<KVT, NT, 64>(p, kmap, vmap, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+bool decode_plan(int batch, int q_len, int num_q_heads, int num_kv_heads, int block_size,
+                 int max_context_len, DecodePlan *plan)
+{
+    if (batch <= 0 || q_len <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads)
+        return false;
+    const int group = num_q_heads / num_kv_heads;
+    const int rows = q_len * group;
+    plan->nt = rows <= 8 ? 1 : 2;
+    plan->rows_per_cta = 8 * plan->nt;
+    plan->row_groups = (rows + plan->rows_per_cta - 1) / plan->rows_per_cta;
+    const int max_blocks = (max_context_len + block_size - 1) / block_size;
+    const long long units = (long long)batch * num_kv_heads * plan->row_groups;
+    // Aim for about `ctas_per_sm` resident CTAs on every SM in a single wave;
+    // never split below one block per warp.
+    int ctas_per_sm = 2;
+    if (const char *env = getenv("PKVQ_DECODE_CTAS_PER_SM")) {
+        const int v = atoi(env);
+        if (v >= 1 && v <= 16)
+            ctas_per_sm = v;
+    }
+    const long long target = (long long)ctas_per_sm * device_sm_count();
+    long long splits = (target + units - 1) / units;
+    const long long max_splits = max(1, (max_blocks + kWarps - 1) / kWarps);
+    splits = max(1LL, min(splits, max_splits));
+    int bps = max_blocks > 0 ? (int)((max_blocks + splits - 1) / splits) : 1;
+    splits = max_blocks > 0 ? (max_blocks + bps - 1) / bps : 1;
+    plan->num_splits = (int)splits;
+    plan->blocks_per_split = bps;
+    plan->workspace_bytes =
+        splits > 1 ? (size_t)batch * num_kv_heads * splits * rows * (kHeadDim + 2) * sizeof(float)
+                   : 0;
+    return true;
+}
+
+cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_dtype,
+                          const CUtensorMap &kmap, const CUtensorMap &vmap, cudaStream_t stream)
+{
+    cudaError_t e;
+    if (kv_dtype == kKvFp8)
+        e = plan.nt == 1 ? launch_bs<kKvFp8, 1>(p, kmap, vmap, stream)
+                         : launch_bs<kKvFp8, 2>(p, kmap, vmap, stream);
+    else
+        e = plan.nt == 1 ? launch_bs<kKvInt8, 1>(p, kmap, vmap, stream)
+                         : launch_bs<kKvInt8, 2>(p, kmap, vmap, stream);
+    if (e != cudaSuccess || p.num_splits == 1)
+        return e;
+    const long long rows_total = (long long)p.batch * p.num_kv_heads * p.rows;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((rows_total + 3) / 4));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_merge_kernel, p);
+}
+
+}  // namespace pkvq

@@ -1,0 +1,167 @@
+"""Helpers shared by the GPU parity tests: build the same seeded case on the
+GPU (through the C ABI) and in the CPU oracle, and compare."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import paged_quantized_kv_quant_b200 as pk
+import synth
+
+# Output tolerance: fp16 outputs vs the FP64 oracle, FP32 accumulation.
+MAX_ABS_TOL = 2e-3
+REL_L2_TOL = 1e-3
+LSE_TOL = 2e-3
+
+NAN_E4M3 = 0x7F          # an E4M3 NaN code: fills never-written cache slots
+NAN_FP16_BITS = 0x7E00
+
+
+def bits16(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def oracle_cache(case: synth.Case) -> oracle.Cache:
+    s = case.spec
+    c = oracle.Cache(s.kv_dtype, case.num_blocks, s.block_size, s.num_kv_heads, s.head_dim,
+                     None if case.k_scale is None else case.k_scale.numpy(),
+                     None if case.v_scale is None else case.v_scale.numpy())
+    c.write(bits16(case.k), bits16(case.v), case.slot_mapping.numpy())
+    return c
+
+
+def gpu_cache(case: synth.Case, poison: bool = True, write: bool = True) -> pk.PagedKVCache:
+    """Allocates the cache on the GPU, fills every slot with NaN patterns
+    (so that reading a never-written slot would show), then writes all
+    cached tokens through pkvq_kv_write_quant."""
+    s = case.spec
+    cache = pk.PagedKVCache.allocate(s.kv_dtype, case.num_blocks, s.block_size,
+                                     s.num_kv_heads, s.head_dim, k_scale=case.k_scale,
+                                     v_scale=case.v_scale)
+    if poison:
+        cache.k_cache.fill_(NAN_E4M3)
+        cache.v_cache.fill_(NAN_E4M3)
+        if cache.k_scale_tok is not None:
+            cache.k_scale_tok.view(torch.int16).fill_(NAN_FP16_BITS)
+            cache.v_scale_tok.view(torch.int16).fill_(NAN_FP16_BITS)
+    if write and case.k.shape[0]:
+        pk.kv_write_quant(cache, case.k.cuda(), case.v.cuda(), case.slot_mapping.cuda())
+    return cache
+
+
+def written_mask(case: synth.Case) -> np.ndarray:
+    """[NB][bs] bool: slots that hold a cached token."""
+    s = case.spec
+    m = np.zeros((case.num_blocks, s.block_size), bool)
+    sm = case.slot_mapping.numpy()
+    sm = sm[sm >= 0]
+    m[sm // s.block_size, sm % s.block_size] = True
+    return m
+
+
+def assert_codes_equal(cache: pk.PagedKVCache, oc: oracle.Cache, case: synth.Case) -> None:
+    """Bit-exact comparison of every written slot's codes (and INT8 scales)."""
+    m = written_mask(case)
+    for name in ("k_cache", "v_cache"):
+        g = getattr(cache, name).cpu().numpy()
+        o = getattr(oc, name)
+        gw = g.transpose(0, 2, 1, 3)[m]
+        ow = o.transpose(0, 2, 1, 3)[m]
+        bad = np.nonzero(gw != ow)
+        assert gw.shape == ow.shape
+        assert bad[0].size == 0, f"{name}: {bad[0].size} codes differ, first at {bad}"
+    if case.spec.kv_dtype == synth.INT8:
+        for name in ("k_scale_tok", "v_scale_tok"):
+            g = bits16(getattr(cache, name).cpu()).transpose(0, 2, 1)[m]
+            o = getattr(oc, name).transpose(0, 2, 1)[m]
+            assert np.array_equal(g, o), f"{name} differs"
+
+
+def run_gpu(case: synth.Case, cache: pk.PagedKVCache, want_lse: bool = True):
+    s = case.spec
+    dev = "cuda"
+    bt = case.block_table.to(dev)
+    ctx = case.context_lens.to(dev)
+    if s.kind == "decode":
+        B = len(s.context_lens)
+        ql = s.q_lens[0]
+        q = case.q.view(B, ql, s.num_q_heads, s.head_dim).to(dev)
+        lse = torch.empty((B, ql, s.num_q_heads), dtype=torch.float32, device=dev) \
+            if want_lse else None
+        out = pk.paged_attn_decode(cache, q, bt, ctx, max(s.context_lens + [0]),
+                                   case.softmax_scale, lse=lse)
+        out = out.view(-1, s.num_q_heads, s.head_dim)
+        lse = None if lse is None else lse.view(-1, s.num_q_heads)
+    else:
+        q = case.q.to(dev)
+        lse = torch.empty((q.shape[0], s.num_q_heads), dtype=torch.float32, device=dev) \
+            if want_lse else None
+        out = pk.paged_attn_prefill(cache, q, case.cu_seqlens_q.to(dev), bt, ctx,
+                                    max(s.q_lens + [0]), case.softmax_scale, lse=lse)
+    torch.cuda.synchronize()
+    return out.cpu(), (None if lse is None else lse.cpu())
+
+
+def run_oracle(case: synth.Case, oc: oracle.Cache, rows=None):
+    return oracle.paged_attention(oc, bits16(case.q), case.cu_seqlens_q.numpy(),
+                                  case.context_lens.numpy(), case.block_table.numpy(),
+                                  case.softmax_scale, rows=rows)[:2]
+
+
+def row_vmax(case: synth.Case, oc: oracle.Cache) -> np.ndarray:
+    """[total_q][Hq]: largest |dequantised V| over the keys each row sees."""
+    s = case.spec
+    G = s.num_q_heads // s.num_kv_heads
+    bt = case.block_table.numpy()
+    cu = case.cu_seqlens_q.numpy()
+    out = np.zeros((int(cu[-1]), s.num_q_heads))
+    for b, (c, ql) in enumerate(zip(s.context_lens, s.q_lens)):
+        if c == 0:
+            continue
+        j = np.arange(c)
+        blk, off = bt[b, j // s.block_size], j % s.block_size
+        codes = oc.v_cache[blk, :, off, :]                      # [c][Hkv][D]
+        if s.kv_dtype == synth.FP8_E4M3:
+            v = oracle.e4m3_decode(codes) * oc.v_scale.astype(np.float64)[None, :, None]
+        else:
+            sc = oc.v_scale_tok[blk, :, off].view(np.float16).astype(np.float64)
+            v = codes.view(np.int8).astype(np.float64) * sc[:, :, None]
+        pre = np.maximum.accumulate(np.abs(v).max(-1), axis=0)  # [c][Hkv]
+        for t in range(ql):
+            pos = c - ql + t
+            if pos >= 0:
+                out[cu[b] + t] = np.repeat(pre[pos], G)
+    return out
+
+
+def assert_close(out_gpu: torch.Tensor, ref: np.ndarray, lse_gpu=None, lse_ref=None,
+                 max_abs=MAX_ABS_TOL, rel_l2=REL_L2_TOL, what="", vmax=None):
+    """Strict form (vmax None): the stated bound, max |err| <= 2e-3 and
+    relative L2 <= 1e-3.  With vmax (per-row largest |v| the row sees), the
+    per-element bound adds what fp16 operands and an fp16 output can cost when
+    values are large: 2^-10 * (|o| + vmax) (one fp16 rounding of the output,
+    of P, of the INT8-dequantised V, and of l's mismatch with P)."""
+    g = out_gpu.double().numpy()
+    assert g.shape == ref.shape, (g.shape, ref.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    err = np.abs(g - ref)
+    tol = max_abs
+    if vmax is not None:
+        tol = max_abs + 2.0 ** -10 * (np.abs(ref) + vmax[..., None])
+    over = err - tol
+    mx = float(over.max()) if err.size else -1.0
+    den = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(g - ref) / den) if den > 0 else float(np.linalg.norm(g))
+    at = np.unravel_index(over.argmax(), err.shape) if err.size else None
+    assert mx <= 0, f"{what}: |err| {float(err[at]):.3e} above its bound by {mx:.3e} at {at}"
+    mx = float(err.max()) if err.size else 0.0
+    assert rel <= rel_l2, f"{what}: rel L2 {rel:.3e} > {rel_l2}"
+    if lse_gpu is not None and lse_ref is not None:
+        lg = lse_gpu.double().numpy()
+        fin = np.isfinite(lse_ref)
+        assert np.array_equal(np.isfinite(lg), fin), f"{what}: lse finiteness differs"
+        if fin.any():
+            le = float(np.abs(lg[fin] - lse_ref[fin]).max())
+            assert le <= LSE_TOL, f"{what}: lse err {le:.3e}"
+    return mx, rel

@@ -1,0 +1,142 @@
+"""GPU parity of pkvq_paged_attn_decode against the FP64 oracle on small and
+ragged shapes, covering the numerical bug classes the 1Cat-LLM README lists
+for its kernels ("Layer 2": short-chunk causal visibility, missed score
+maxima, overflowing score tiles, tail range)."""
+import numpy as np
+import pytest
+import torch
+
+import paged_quantized_kv_quant_b200 as pk
+import synth
+from pkvq_testutil import (assert_close, assert_codes_equal, gpu_cache, oracle_cache, row_vmax,
+                           run_gpu, run_oracle)
+
+pytestmark = pytest.mark.gpu
+
+FP8, INT8 = synth.FP8_E4M3, synth.INT8
+
+CASES = [
+    # dtype, Hq, Hkv, ctx list, q_len, bs
+    (FP8, 8, 2, [1024], 1, 16),             # workload 1 shape
+    (FP8, 32, 4, [777, 16, 1, 2049], 1, 16),  # ragged tails, one-key context
+    (FP8, 4, 4, [100, 35], 1, 16),          # MHA (G = 1)
+    (FP8, 16, 1, [513], 1, 32),             # G = 16 -> two row tiles
+    (FP8, 8, 4, [300, 129], 1, 64),
+    (INT8, 32, 4, [999, 17], 5, 16),        # verify: q_len 5 -> 40 rows, row groups
+    (INT8, 8, 2, [5, 6, 300], 5, 16),       # q_len == context: first row sees 1 key
+    (INT8, 16, 4, [64, 65], 3, 32),
+    (FP8, 8, 1, [4099], 4, 16),             # q_len 4, G 8 -> 32 rows
+    (FP8, 32, 4, [16384], 1, 16),           # long: many splits
+    (INT8, 8, 2, [20000, 3], 2, 16),
+]
+
+
+def _case(dtype, Hq, Hkv, ctx, ql, bs, seed=0, **kw):
+    spec = synth.CaseSpec("decode", dtype, Hq, Hkv, list(ctx), [ql] * len(ctx),
+                          block_size=bs, seed=seed, **kw)
+    return synth.make_case(spec)
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,ctx,ql,bs", CASES)
+def test_decode_matches_oracle(dtype, Hq, Hkv, ctx, ql, bs):
+    case = _case(dtype, Hq, Hkv, ctx, ql, bs, seed=21, outlier_frac=0.01)
+    cache = gpu_cache(case)
+    oc = oracle_cache(case)
+    assert_codes_equal(cache, oc, case)
+    out, lse = run_gpu(case, cache)
+    ref, ref_lse = run_oracle(case, oc)
+    assert_close(out, ref, lse, ref_lse, what=f"decode {dtype} {Hq}/{Hkv} {ctx} q{ql} bs{bs}",
+                 vmax=row_vmax(case, oc))
+    assert pk.device_status() == 0
+
+
+def test_decode_empty_context_and_q_len_beyond_context():
+    # context 0 -> zeros / -inf; q_len 3 over context 2 -> the first row sees nothing
+    case = _case(FP8, 8, 2, [0, 2, 40], 3, 16, seed=4)
+    case.spec.context_lens = [0, 2, 40]
+    cache = gpu_cache(case)
+    oc = oracle_cache(case)
+    out, lse = run_gpu(case, cache)
+    ref, ref_lse = run_oracle(case, oc)
+    assert np.all(out[:3].numpy() == 0)
+    assert np.all(np.isneginf(lse[:3].numpy()))
+    assert np.all(out[3].numpy() == 0) and np.all(np.isneginf(lse[3].numpy()))
+    assert_close(out, ref, lse, ref_lse, what="empty rows",
+                 vmax=row_vmax(case, oc))
+
+
+def test_decode_max_in_last_tile_and_large_logits():
+    case = _case(FP8, 8, 2, [3000, 1500], 1, 16, seed=5)
+    # a key at the very end of each context that aligns with every query:
+    # the softmax maximum sits in the last (partial) tile
+    for s, c in enumerate(case.spec.context_lens):
+        j = int(case.token_offsets[s]) + c - 1
+        case.k[j] = (case.q[s].float().view(2, 4, 128).mean(1) * 3).to(torch.float16)
+    case.q.mul_(40.0)        # logits in the hundreds: scores must not overflow
+    case.k_scale = synth.per_head_absmax_scale(case.k)
+    cache = gpu_cache(case)
+    oc = oracle_cache(case)
+    out, lse = run_gpu(case, cache)
+    ref, ref_lse = run_oracle(case, oc)
+    assert_close(out, ref, lse, ref_lse, what="peaked",
+                 vmax=row_vmax(case, oc))
+
+
+def test_decode_uniform_logits_mean_of_values():
+    case = _case(FP8, 8, 2, [513], 1, 16, seed=6)
+    case.q.zero_()
+    cache = gpu_cache(case)
+    oc = oracle_cache(case)
+    out, lse = run_gpu(case, cache)
+    ref, ref_lse = run_oracle(case, oc)
+    assert_close(out, ref, lse, ref_lse, what="uniform",
+                 vmax=row_vmax(case, oc))
+    assert np.allclose(lse.numpy(), np.log(513), atol=1e-4)
+
+
+def test_decode_block_table_permutation_is_bitwise_invariant():
+    case = _case(INT8, 16, 4, [700, 333], 2, 16, seed=7)
+    cache = gpu_cache(case)
+    out1, lse1 = run_gpu(case, cache)
+    # move every block to a new physical id
+    perm = torch.randperm(case.num_blocks, generator=torch.Generator().manual_seed(3))
+    moved = pk.PagedKVCache(cache.dtype, torch.empty_like(cache.k_cache),
+                            torch.empty_like(cache.v_cache),
+                            k_scale_tok=torch.empty_like(cache.k_scale_tok),
+                            v_scale_tok=torch.empty_like(cache.v_scale_tok))
+    pd = perm.cuda()
+    moved.k_cache[pd] = cache.k_cache
+    moved.v_cache[pd] = cache.v_cache
+    moved.k_scale_tok[pd] = cache.k_scale_tok
+    moved.v_scale_tok[pd] = cache.v_scale_tok
+    case.block_table = perm[case.block_table.long()].to(torch.int32)
+    out2, lse2 = run_gpu(case, moved)
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
+
+
+def test_decode_causal_append_within_tolerance():
+    # the same prefix decoded at two context lengths: the shorter run's answer
+    # for its last token matches the oracle either way (split plans differ)
+    case = _case(FP8, 8, 2, [2000], 1, 16, seed=8)
+    cache = gpu_cache(case)
+    oc = oracle_cache(case)
+    for c in (1999, 2000):
+        case.spec.context_lens = [c]
+        case.context_lens = torch.tensor([c], dtype=torch.int32)
+        out, lse = run_gpu(case, cache)
+        ref, ref_lse = run_oracle(case, oc)
+        assert_close(out, ref, lse, ref_lse, what=f"ctx {c}",
+                 vmax=row_vmax(case, oc))
+
+
+def test_decode_workspace_too_small_is_rejected():
+    case = _case(FP8, 32, 4, [8192], 1, 16, seed=9)
+    cache = gpu_cache(case)
+    need = pk.decode_workspace_bytes(cache, 1, 1, 32, 8192)
+    assert need > 0
+    q = case.q.view(1, 1, 32, 128).cuda()
+    ws = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(pk.PkvqError) as e:
+        pk.paged_attn_decode(cache, q, case.block_table.cuda(), case.context_lens.cuda(), 8192,
+                             case.softmax_scale, workspace=ws)
+    assert e.value.status == 4
