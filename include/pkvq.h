@@ -144,6 +144,27 @@ PKVQ_API pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void 
                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Decode without a caller-provided workspace.  The pages have no counterpart:
+ * this is an addition for callers that cannot allocate device memory (for
+ * example an engine whose caching allocator already holds nearly all of HBM,
+ * or a plugin whose host framework owns every allocation).
+ * Same arguments, results and errors as pkvq_paged_attn_decode, minus the
+ * workspace: the split-KV scratch is a fixed 8 MiB array compiled into the
+ * library (held on every GPU that loads it, until exit).  Nothing is
+ * allocated.  Shapes whose workspace (pkvq_decode_workspace_bytes) exceeds
+ * 8 MiB return PKVQ_ERR_WORKSPACE_TOO_SMALL.  The first call on each device
+ * looks up the array's device address; make that first call before any
+ * stream capture.  All calls on a device share the array: calls that may
+ * overlap on the device race and must be ordered by the caller.  The array
+ * needs no clearing between calls.
+ */
+PKVQ_API pkvq_status pkvq_paged_attn_decode_noalloc(const pkvq_cache *cache, const void *q,
+                                   void *out, float *lse_out, const int32_t *block_table,
+                                   int32_t max_blocks_per_seq, const int32_t *context_lens,
+                                   int32_t batch, int32_t q_len, int32_t num_q_heads,
+                                   int32_t max_context_len, float softmax_scale, void *stream);
+
+/*
  * Causal (chunked) prefill over a cached prefix, varlen batch.
  * Source: "1Cat-LLM" README, "Layer 2" (causal online softmax with FP32
  * accumulation, prefix / causal-tail separation, wide QK/PV tensor-core

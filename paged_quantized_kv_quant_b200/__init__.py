@@ -31,6 +31,7 @@ EXPORTED = (
     "pkvq_kv_write_quant",
     "pkvq_decode_workspace_bytes",
     "pkvq_paged_attn_decode",
+    "pkvq_paged_attn_decode_noalloc",
     "pkvq_paged_attn_prefill",
     "pkvq_status_string",
     "pkvq_device_status",
@@ -81,6 +82,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pkvq_paged_attn_decode.restype = I32
     lib.pkvq_paged_attn_decode.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, I32,
                                            ctypes.c_float, P, SZ, P]
+    lib.pkvq_paged_attn_decode_noalloc.restype = I32
+    lib.pkvq_paged_attn_decode_noalloc.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, I32,
+                                                   ctypes.c_float, P]
     lib.pkvq_paged_attn_prefill.restype = I32
     lib.pkvq_paged_attn_prefill.argtypes = [P, P, P, P, P, P, I32, P, I32, I32, I32,
                                             ctypes.c_float, P, SZ, P]
