@@ -347,13 +347,13 @@ pkvq_status pkvq_paged_attn_prefill(const pkvq_cache *cache, const void *q, void
     p.group = group;
     p.num_blocks = cache->num_blocks;
     p.block_size = cache->block_size;
-    p.tokens_per_tile = 128 / group;
+    p.tokens_per_tile = 128 / group;   // 128 query rows per CTA
     p.q_tiles = (max_q_len + p.tokens_per_tile - 1) / p.tokens_per_tile;
     p.scale_log2 = softmax_scale * kLog2e;
     p.status = status_ptr();
     if (!p.status)
         return PKVQ_ERR_CUDA;
-    return from_cuda(launch_prefill(p, cache->dtype, km, vm, static_cast<cudaStream_t>(stream)));
+    return from_cuda(launch_prefill_tc(p, cache->dtype, km, vm, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

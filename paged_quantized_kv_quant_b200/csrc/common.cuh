@@ -177,6 +177,31 @@ __device__ __forceinline__ uint32_t e4m3x2_to_half2(uint32_t pair)
     return out;
 }
 
+// Four E4M3 codes (bytes b0..b3 of x) -> half2 (b0, b1) and half2 (b2, b3).
+__device__ __forceinline__ void e4m3x4_to_half2x2(uint32_t x, uint32_t &lo, uint32_t &hi)
+{
+    asm("{\n\t.reg .b16 a, b;\n\t"
+        "mov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(x));
+}
+
+// Four int8 codes (bytes b0..b3 of x) -> half2 (b0, b1) and half2 (b2, b3),
+// exact (see s8x2_to_half2).
+__device__ __forceinline__ void s8x4_to_half2x2(uint32_t x, uint32_t &lo, uint32_t &hi)
+{
+    const uint32_t biased = x ^ 0x80808080u;
+    uint32_t l = __byte_perm(biased, 0x64646464u, 0x5140);
+    uint32_t h = __byte_perm(biased, 0x64646464u, 0x7362);
+    const __half2 k = __half2half2(__ushort_as_half(0x6480));   // 1152
+    __half2 lh = __hsub2(*reinterpret_cast<__half2 *>(&l), k);
+    __half2 hh = __hsub2(*reinterpret_cast<__half2 *>(&h), k);
+    lo = *reinterpret_cast<uint32_t *>(&lh);
+    hi = *reinterpret_cast<uint32_t *>(&hh);
+}
+
 // Two signed int8 codes (bytes b0, b1 of `pair`) -> exact half2 values.
 // 0x6400 | (c ^ 0x80) is the fp16 number 1024 + 128 + c; subtracting 1152
 // is exact for |c| <= 128.

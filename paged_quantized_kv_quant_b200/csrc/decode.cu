@@ -42,11 +42,17 @@ constexpr float kLn2 = 0.693147180559945309f;
 
 template <int BS>
 struct DecodeCfg {
+#ifdef PKVQ_DECODE_STAGES
+    static constexpr int kStages = BS == 16 ? PKVQ_DECODE_STAGES : (BS == 32 ? 3 : 2);
+#else
     static constexpr int kStages = BS == 16 ? 4 : (BS == 32 ? 3 : 2);
+#endif
+    static constexpr int kUnroll = BS == 16 ? 2 : 1;   // cache blocks per loop iteration
     static constexpr int kTileBytes = BS * 128;
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kScaleHalves = 2 * BS;     // K then V scales of one block
     static constexpr int kMT = BS / 16;             // 16-key m-tiles per block
+    static_assert(kStages >= 2 * kUnroll, "ring must hold two iterations");
 };
 
 template <int BS>
@@ -63,12 +69,12 @@ __device__ __forceinline__ uint4 lds128(const uint8_t *p)
 }
 
 template <int KVT>
-__device__ __forceinline__ uint32_t cvt2(uint32_t pair)
+__device__ __forceinline__ void cvt4(uint32_t x, uint32_t &lo, uint32_t &hi)
 {
     if constexpr (KVT == kKvFp8)
-        return e4m3x2_to_half2(pair);
+        e4m3x4_to_half2x2(x, lo, hi);
     else
-        return s8x2_to_half2(pair);
+        s8x4_to_half2x2(x, lo, hi);
 }
 
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b)
@@ -82,6 +88,110 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i)
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
 }
 
+// S^T = K Q^T for one cache block (MT m-tiles of 16 keys), scaled to log2
+// units.  Lane (g, t) reads 32 contiguous code bytes of keys g and g+8 of each
+// m-tile; the swizzled 16-byte chunk c of row r sits at c ^ (r & 7).
+template <int KVT, int NT, int MT>
+__device__ __forceinline__ void qk_block(const uint8_t *kt, const uint16_t *st, int g, int t,
+                                         const uint32_t (&qf)[NT][8][2], float kfac,
+                                         float (&sc)[MT][NT][4])
+{
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int r0 = mt * 16 + g;   // rows r0, r0 + 8 share (row & 7) == g
+        const uint4 ka0 = lds128(kt + r0 * 128 + (((2 * t) ^ g) << 4));
+        const uint4 ka1 = lds128(kt + r0 * 128 + (((2 * t + 1) ^ g) << 4));
+        const uint4 kb0 = lds128(kt + (r0 + 8) * 128 + (((2 * t) ^ g) << 4));
+        const uint4 kb1 = lds128(kt + (r0 + 8) * 128 + (((2 * t + 1) ^ g) << 4));
+        const uint32_t wa[8] = {ka0.x, ka0.y, ka0.z, ka0.w, ka1.x, ka1.y, ka1.z, ka1.w};
+        const uint32_t wb[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                sc[mt][nt][c] = 0.0f;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            uint32_t a[4];
+            cvt4<KVT>(wa[ks], a[0], a[2]);   // key g:   d = 32t+4ks+{0,1} | {2,3}
+            cvt4<KVT>(wb[ks], a[1], a[3]);   // key g+8
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                mma_f16_16816(sc[mt][nt], a, qf[nt][ks]);
+        }
+        float f0 = kfac, f1 = kfac;
+        if constexpr (KVT == kKvInt8) {
+            f0 *= __half2float(__ushort_as_half(st[r0]));
+            f1 *= __half2float(__ushort_as_half(st[r0 + 8]));
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            sc[mt][nt][0] *= f0, sc[mt][nt][1] *= f0;
+            sc[mt][nt][2] *= f1, sc[mt][nt][3] *= f1;
+        }
+    }
+}
+
+// O^T += V^T P^T for one cache block.  Lane (g, t) reads the 16-byte chunk g
+// (d = 16g .. 16g+15) of keys 2t, 2t+1, 2t+8, 2t+9 of each m-tile; one byte
+// permute pairs two keys' codes for two d rows at once.
+template <int KVT, int NT, int MT, int BS>
+__device__ __forceinline__ void pv_block(const uint8_t *vt, const uint16_t *st, int g, int t,
+                                         int key0, int ctx, const float (&pr)[MT][NT][4],
+                                         float (&o)[NT][8][4])
+{
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        uint32_t pb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            pb[nt][0] = movmatrix_trans(pack_half2(pr[mt][nt][0], pr[mt][nt][1]));
+            pb[nt][1] = movmatrix_trans(pack_half2(pr[mt][nt][2], pr[mt][nt][3]));
+        }
+        const int r0 = mt * 16 + 2 * t;   // key rows r0, r0+1, r0+8, r0+9
+        uint4 v0 = lds128(vt + r0 * 128 + ((g ^ (r0 & 7)) << 4));
+        uint4 v1 = lds128(vt + (r0 + 1) * 128 + ((g ^ ((r0 + 1) & 7)) << 4));
+        uint4 v2 = lds128(vt + (r0 + 8) * 128 + ((g ^ ((r0 + 8) & 7)) << 4));
+        uint4 v3 = lds128(vt + (r0 + 9) * 128 + ((g ^ ((r0 + 9) & 7)) << 4));
+        uint32_t s01 = 0u, s23 = 0u;
+        if constexpr (KVT == kKvInt8) {
+            s01 = (uint32_t)st[BS + r0] | ((uint32_t)st[BS + r0 + 1] << 16);
+            s23 = (uint32_t)st[BS + r0 + 8] | ((uint32_t)st[BS + r0 + 9] << 16);
+        }
+        if (key0 + BS > ctx) {
+            // Slots past the context were never written: their codes (and
+            // INT8 scales) may be NaN patterns, and 0 * NaN would poison O.
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            const int k0 = key0 + r0;
+            if (k0 >= ctx) v0 = z, s01 &= 0xffff0000u;
+            if (k0 + 1 >= ctx) v1 = z, s01 &= 0x0000ffffu;
+            if (k0 + 8 >= ctx) v2 = z, s23 &= 0xffff0000u;
+            if (k0 + 9 >= ctx) v3 = z, s23 &= 0x0000ffffu;
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const uint32_t x0 = word_of(v0, w), x1 = word_of(v1, w);
+            const uint32_t x2 = word_of(v2, w), x3 = word_of(v3, w);
+#pragma unroll
+            for (int hw = 0; hw < 2; ++hw) {   // d-tile dt = 2w + hw: bytes 4w+2hw, 4w+2hw+1
+                const uint32_t sel = hw ? 0x7362u : 0x5140u;
+                uint32_t a[4];
+                cvt4<KVT>(__byte_perm(x0, x1, sel), a[0], a[1]);
+                cvt4<KVT>(__byte_perm(x2, x3, sel), a[2], a[3]);
+                if constexpr (KVT == kKvInt8) {
+                    a[0] = hmul2_u32(a[0], s01);
+                    a[1] = hmul2_u32(a[1], s01);
+                    a[2] = hmul2_u32(a[2], s23);
+                    a[3] = hmul2_u32(a[3], s23);
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+                    mma_f16_16816(o[nt][2 * w + hw], a, pb[nt]);
+            }
+        }
+    }
+}
+
 template <int KVT, int NT, int BS>
 __global__ void __launch_bounds__(kThreads)
 decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -89,6 +199,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 {
     using C = DecodeCfg<BS>;
     constexpr int S = C::kStages;
+    constexpr int U = C::kUnroll;
     constexpr int RC = 8 * NT;
     constexpr int MT = C::kMT;
 
@@ -106,20 +217,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
 
-    // Let the merge kernel (programmatic dependent launch) get scheduled early;
-    // it still waits for this grid to finish before reading the workspace.
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-    if (device_wait_failed(p.status))
-        return;
-    const int ctx = p.context_lens[b];
-    const int nblk_seq = (ctx + BS - 1) / BS;
-    const int blk_begin = split * p.blocks_per_split;
-    if (p.num_splits > 1 && blk_begin >= nblk_seq)
-        return;   // the merge kernel only reads splits that hold keys
-    const int nblk = max(0, min(nblk_seq, blk_begin + p.blocks_per_split) - blk_begin);
-    const int n_it = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
-
+    // Prologue that reads no input: it may overlap the previous kernel in the
+    // stream (this kernel is launched with programmatic dependent launch).
     uint64_t *my_bars = bars + warp * S;
     uint8_t *my_tiles = tiles + warp * S * C::kStageBytes;
     uint16_t *my_scales = scales + warp * S * C::kScaleHalves;
@@ -132,6 +231,29 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
         fence_mbar_init();
     }
     __syncwarp();
+    // Inputs may come from the previous kernel: wait for it to complete.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // Let the merge kernel get scheduled early; it still waits for this grid
+    // to finish before reading the workspace.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    if (device_wait_failed(p.status))
+        return;
+    const int blk_begin = split * p.blocks_per_split;
+    // Block ids of this warp's first 64 iterations are loaded speculatively
+    // (every index stays inside the table row), in parallel with the context
+    // length, so the first copies wait for one memory round trip, not two.
+    const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq;
+    auto lblk = [&](int it) { return blk_begin + warp + kWarps * it; };
+    int win0 = lblk(lane) < p.max_blocks_per_seq ? __ldg(bt + lblk(lane)) : 0;
+    int win1 = lblk(32 + lane) < p.max_blocks_per_seq ? __ldg(bt + lblk(32 + lane)) : 0;
+    int win_base = 0;
+    const int ctx = p.context_lens[b];
+    const int nblk_seq = (ctx + BS - 1) / BS;
+    if (p.num_splits > 1 && blk_begin >= nblk_seq)
+        return;   // the merge kernel only reads splits that hold keys
+    const int nblk = max(0, min(nblk_seq, blk_begin + p.blocks_per_split) - blk_begin);
+    const int n_it = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
 
     // ---- query fragments (B operand of S^T = K Q^T), loop invariant ----
     const int h0 = h * p.group;
@@ -186,11 +308,6 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     }
 
     // ---- block ids: a sliding window of 64 iterations held in two registers ----
-    const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq;
-    auto lblk = [&](int it) { return blk_begin + warp + kWarps * it; };
-    int win0 = lane < n_it ? __ldg(bt + lblk(lane)) : 0;
-    int win1 = 32 + lane < n_it ? __ldg(bt + lblk(32 + lane)) : 0;
-    int win_base = 0;
 
     constexpr uint32_t kTx = C::kStageBytes + (KVT == kKvInt8 ? C::kScaleHalves * 2 : 0);
     auto issue = [&](int j) {   // warp-uniform call
@@ -226,76 +343,62 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     const int min_pos = ctx - p.q_len;
     int it = 0;
     bool ok = true;
-    for (; it < n_it; ++it) {
-        const int stage = it % S;
-        if (!mbar_wait(&my_bars[stage], (it / S) & 1, p.status)) {
-            ok = false;
+    for (; it < n_it; it += U) {
+        // ---- wait for this iteration's U blocks ----
+        bool have[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            have[u] = it + u < n_it;
+            if (have[u] && !mbar_wait(&my_bars[(it + u) % S], ((it + u) / S) & 1, p.status))
+                ok = false;
+        }
+        if (!ok)
             break;
-        }
-        const uint8_t *kt = my_tiles + stage * C::kStageBytes;
-        const uint8_t *vt = kt + C::kTileBytes;
-        const uint16_t *st = my_scales + stage * C::kScaleHalves;
-        const int key0 = lblk(it) * BS;
 
-        // ---------------- S^T = K Q^T ----------------
-        float sc[MT][NT][4];
+        // ---- S^T = K Q^T, masked ----
+        float sc[U][MT][NT][4];
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            const int r0 = mt * 16 + g;   // key rows r0 and r0 + 8; (row & 7) == g
-            const uint4 ka0 = lds128(kt + r0 * 128 + (((2 * t) ^ g) << 4));
-            const uint4 ka1 = lds128(kt + r0 * 128 + (((2 * t + 1) ^ g) << 4));
-            const uint4 kb0 = lds128(kt + (r0 + 8) * 128 + (((2 * t) ^ g) << 4));
-            const uint4 kb1 = lds128(kt + (r0 + 8) * 128 + (((2 * t + 1) ^ g) << 4));
-            const uint32_t wa[8] = {ka0.x, ka0.y, ka0.z, ka0.w, ka1.x, ka1.y, ka1.z, ka1.w};
-            const uint32_t wb[8] = {kb0.x, kb0.y, kb0.z, kb0.w, kb1.x, kb1.y, kb1.z, kb1.w};
+        for (int u = 0; u < U; ++u) {
+            const int stage = (it + u) % S;
+            const uint8_t *kt = my_tiles + stage * C::kStageBytes;
+            const uint16_t *st = my_scales + stage * C::kScaleHalves;
+            if (have[u]) {
+                qk_block<KVT, NT, MT>(kt, st, g, t, qf, kfac, sc[u]);
+                const int key0 = lblk(it + u) * BS;
+                if (key0 + BS - 1 > min_pos) {   // a key may lie past a row's position
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
+                    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    sc[mt][nt][c] = 0.0f;
+                        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t a[4] = {cvt2<KVT>(wa[ks] & 0xffffu), cvt2<KVT>(wb[ks] & 0xffffu),
-                                       cvt2<KVT>(wa[ks] >> 16), cvt2<KVT>(wb[ks] >> 16)};
+                            for (int c = 0; c < 4; ++c) {
+                                const int key = key0 + mt * 16 + g + (c >> 1) * 8;
+                                if (key > pos[nt][c & 1])
+                                    sc[u][mt][nt][c] = -INFINITY;
+                            }
+                }
+            } else {
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                    mma_f16_16816(sc[mt][nt], a, qf[nt][ks]);
-            }
-            float f0 = kfac, f1 = kfac;
-            if constexpr (KVT == kKvInt8) {
-                f0 *= __half2float(__ushort_as_half(st[r0]));
-                f1 *= __half2float(__ushort_as_half(st[r0 + 8]));
-            }
+                for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                sc[mt][nt][0] *= f0, sc[mt][nt][1] *= f0;
-                sc[mt][nt][2] *= f1, sc[mt][nt][3] *= f1;
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            sc[u][mt][nt][c] = -INFINITY;
             }
         }
 
-        // causal / context mask, only where a key can lie past a row's position
-        if (key0 + BS - 1 > min_pos) {
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int key = key0 + mt * 16 + g + (c >> 1) * 8;
-                        if (key > pos[nt][c & 1])
-                            sc[mt][nt][c] = -INFINITY;
-                    }
-        }
-
-        // ---------------- online softmax (base 2) ----------------
+        // ---- online softmax (base 2) over the U blocks ----
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 float mx = -INFINITY;
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt)
-                    mx = fmaxf(mx, fmaxf(sc[mt][nt][i], sc[mt][nt][2 + i]));
+                for (int u = 0; u < U; ++u)
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt)
+                        mx = fmaxf(mx, fmaxf(sc[u][mt][nt][i], sc[u][mt][nt][2 + i]));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
@@ -303,86 +406,52 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
                 const float m_use = m_new == -INFINITY ? 0.0f : m_new;
                 const float corr = fast_exp2(m[nt][i] - m_use);
                 m[nt][i] = m_new;
-                float ls = l[nt][i] * corr;
+                if (__any_sync(0xffffffffu, corr != 1.0f)) {
+                    l[nt][i] *= corr;
 #pragma unroll
-                for (int dt = 0; dt < 8; ++dt) {
-                    o[nt][dt][i] *= corr;
-                    o[nt][dt][2 + i] *= corr;
+                    for (int dt = 0; dt < 8; ++dt) {
+                        o[nt][dt][i] *= corr;
+                        o[nt][dt][2 + i] *= corr;
+                    }
                 }
+                float ls = 0.0f;
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    const float p0 = fast_exp2(sc[mt][nt][i] - m_use);
-                    const float p1 = fast_exp2(sc[mt][nt][2 + i] - m_use);
-                    sc[mt][nt][i] = p0;
-                    sc[mt][nt][2 + i] = p1;
-                    ls += p0 + p1;
-                }
-                l[nt][i] = ls;
+                for (int u = 0; u < U; ++u)
+#pragma unroll
+                    for (int mt = 0; mt < MT; ++mt) {
+                        const float p0 = fast_exp2(sc[u][mt][nt][i] - m_use);
+                        const float p1 = fast_exp2(sc[u][mt][nt][2 + i] - m_use);
+                        sc[u][mt][nt][i] = p0;
+                        sc[u][mt][nt][2 + i] = p1;
+                        ls += p0 + p1;
+                    }
+                l[nt][i] += ls;
             }
         }
 
-        // ---------------- O^T += V^T P^T ----------------
+        // ---- O^T += V^T P^T ----
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            uint32_t pb[NT][2];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                pb[nt][0] = movmatrix_trans(pack_half2(sc[mt][nt][0], sc[mt][nt][1]));
-                pb[nt][1] = movmatrix_trans(pack_half2(sc[mt][nt][2], sc[mt][nt][3]));
-            }
-            const int r0 = mt * 16 + 2 * t;   // key rows r0, r0+1, r0+8, r0+9
-            uint4 v0 = lds128(vt + r0 * 128 + ((g ^ (r0 & 7)) << 4));
-            uint4 v1 = lds128(vt + (r0 + 1) * 128 + ((g ^ ((r0 + 1) & 7)) << 4));
-            uint4 v2 = lds128(vt + (r0 + 8) * 128 + ((g ^ ((r0 + 8) & 7)) << 4));
-            uint4 v3 = lds128(vt + (r0 + 9) * 128 + ((g ^ ((r0 + 9) & 7)) << 4));
-            uint32_t s01 = 0u, s23 = 0u;
-            if constexpr (KVT == kKvInt8) {
-                s01 = (uint32_t)st[BS + r0] | ((uint32_t)st[BS + r0 + 1] << 16);
-                s23 = (uint32_t)st[BS + r0 + 8] | ((uint32_t)st[BS + r0 + 9] << 16);
-            }
-            if (key0 + BS > ctx) {
-                // Slots past the context were never written: their codes (and
-                // INT8 scales) may be NaN patterns, and 0 * NaN would poison O.
-                const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-                const int k0 = key0 + r0;
-                if (k0 >= ctx) v0 = z, s01 &= 0xffff0000u;
-                if (k0 + 1 >= ctx) v1 = z, s01 &= 0x0000ffffu;
-                if (k0 + 8 >= ctx) v2 = z, s23 &= 0xffff0000u;
-                if (k0 + 9 >= ctx) v3 = z, s23 &= 0x0000ffffu;
-            }
-#pragma unroll
-            for (int dt = 0; dt < 8; ++dt) {
-                const int wi = dt >> 1;
-                const uint32_t bo = 2u * (dt & 1);
-                const uint32_t x0 = word_of(v0, wi), x1 = word_of(v1, wi);
-                const uint32_t x2 = word_of(v2, wi), x3 = word_of(v3, wi);
-                const uint32_t sel0 = bo | ((4u + bo) << 4);
-                const uint32_t sel1 = (bo + 1u) | ((5u + bo) << 4);
-                uint32_t a[4] = {cvt2<KVT>(__byte_perm(x0, x1, sel0) & 0xffffu),
-                                 cvt2<KVT>(__byte_perm(x0, x1, sel1) & 0xffffu),
-                                 cvt2<KVT>(__byte_perm(x2, x3, sel0) & 0xffffu),
-                                 cvt2<KVT>(__byte_perm(x2, x3, sel1) & 0xffffu)};
-                if constexpr (KVT == kKvInt8) {
-                    a[0] = hmul2_u32(a[0], s01);
-                    a[1] = hmul2_u32(a[1], s01);
-                    a[2] = hmul2_u32(a[2], s23);
-                    a[3] = hmul2_u32(a[3], s23);
-                }
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-                    mma_f16_16816(o[nt][dt], a, pb[nt]);
-            }
+        for (int u = 0; u < U; ++u) {
+            if (!have[u])
+                continue;
+            const int stage = (it + u) % S;
+            const uint8_t *vt = my_tiles + stage * C::kStageBytes + C::kTileBytes;
+            const uint16_t *st = my_scales + stage * C::kScaleHalves;
+            pv_block<KVT, NT, MT, BS>(vt, st, g, t, lblk(it + u) * BS, ctx, sc[u], o);
         }
 
         __syncwarp();
-        if (issued < n_it) {
-            issue(issued);
-            ++issued;
-        }
-        if ((it & 31) == 31) {
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (issued < n_it) {
+                issue(issued);
+                ++issued;
+            }
+        if (it + U >= win_base + 32) {
             win_base += 32;
             win0 = win1;
-            win1 = win_base + 32 + lane < n_it ? __ldg(bt + lblk(win_base + 32 + lane)) : 0;
+            win1 = lblk(win_base + 32 + lane) < p.max_blocks_per_seq
+                       ? __ldg(bt + lblk(win_base + 32 + lane)) : 0;
         }
     }
     if (!ok) {
@@ -467,6 +536,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 
 // Merge of the split partial states (one warp per output row):
 // M = max_i m_i, L = sum_i l_i 2^(m_i - M), O = sum_i O_i 2^(m_i - M) / L.
+// Lane i reads split i's (m, l); the O rows are then read four splits at a
+// time so their loads overlap.
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -483,18 +554,50 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
     const int nvalid = min(p.num_splits, (nblk + p.blocks_per_split - 1) / p.blocks_per_split);
     const size_t base = ((size_t)b * p.num_kv_heads + h) * p.num_splits * p.rows + rr;
     float M = -INFINITY;
-    for (int s = 0; s < nvalid; ++s)
+    for (int s = lane; s < nvalid; s += 32)
         M = fmaxf(M, p.ws_ml[(base + (size_t)s * p.rows) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     const float Mu = M == -INFINITY ? 0.0f : M;
     float L = 0.0f;
     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < nvalid; ++s) {
-        const size_t wrow = base + (size_t)s * p.rows;
-        const float e = fast_exp2(p.ws_ml[wrow * 2] - Mu);
-        L += p.ws_ml[wrow * 2 + 1] * e;
-        const float4 v = reinterpret_cast<const float4 *>(p.ws_o + wrow * kHeadDim)[lane];
-        O.x += v.x * e, O.y += v.y * e, O.z += v.z * e, O.w += v.w * e;
+    for (int s0 = 0; s0 < nvalid; s0 += 32) {
+        // weights of splits s0 .. s0+31, one per lane
+        const int sl = s0 + lane;
+        float e = 0.0f;
+        if (sl < nvalid) {
+            const size_t wrow = base + (size_t)sl * p.rows;
+            e = fast_exp2(p.ws_ml[wrow * 2] - Mu);
+            L += p.ws_ml[wrow * 2 + 1] * e;
+        }
+        const int n = min(32, nvalid - s0);
+        int j = 0;
+        for (; j + 4 <= n; j += 4) {
+            float4 v[4];
+            float w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                w[k] = __shfl_sync(0xffffffffu, e, j + k);
+                v[k] = reinterpret_cast<const float4 *>(
+                    p.ws_o + (base + (size_t)(s0 + j + k) * p.rows) * kHeadDim)[lane];
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                O.x += v[k].x * w[k], O.y += v[k].y * w[k];
+                O.z += v[k].z * w[k], O.w += v[k].w * w[k];
+            }
+        }
+        for (; j < n; ++j) {
+            const float w = __shfl_sync(0xffffffffu, e, j);
+            const float4 v = reinterpret_cast<const float4 *>(
+                p.ws_o + (base + (size_t)(s0 + j) * p.rows) * kHeadDim)[lane];
+            O.x += v.x * w, O.y += v.y * w, O.z += v.z * w, O.w += v.w * w;
+        }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        L += __shfl_xor_sync(0xffffffffu, L, o);
     const float vfac = p.v_scale ? __ldg(p.v_scale + h) : 1.0f;
     const int tq = rr / p.group, gq = rr % p.group;
     const size_t orow = ((size_t)b * p.q_len + tq) * p.num_q_heads + h * p.group + gq;
@@ -517,9 +620,17 @@ cudaError_t launch_split(const DecodeParams &p, const CUtensorMap &kmap, const C
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    dim3 grid(p.num_splits, p.num_kv_heads * p.row_groups, p.batch);
-    kern<<<grid, kThreads, smem, stream>>>(kmap, vmap, p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.num_splits, p.num_kv_heads * p.row_groups, p.batch);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, kmap, vmap, p);
 }
 
 template <int KVT, int NT>

@@ -78,8 +78,8 @@ struct PrefillParams {
     uint32_t *status;
 };
 
-cudaError_t launch_prefill(const PrefillParams &p, int kv_dtype, const CUtensorMap &kmap,
-                           const CUtensorMap &vmap, cudaStream_t stream);
+cudaError_t launch_prefill_tc(const PrefillParams &p, int kv_dtype, const CUtensorMap &kmap,
+                              const CUtensorMap &vmap, cudaStream_t stream);
 
 // Encodes a 2-D uint8 tensor map over a cache: rows of 128 bytes, boxes of
 // box_rows rows, 128-byte swizzle.

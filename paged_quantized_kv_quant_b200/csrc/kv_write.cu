@@ -104,6 +104,10 @@ template <int KVT>
 __global__ void __launch_bounds__(kBlockThreads)
 kv_write_quant_kernel(KvWriteParams p)
 {
+    // The next kernel (e.g. decode, launched with programmatic dependent
+    // launch) may start its input-free prologue now; it waits for this grid to
+    // finish before it reads anything.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int row = blockIdx.x * kRowsPerBlock + threadIdx.x / kThreadsPerRow;
     const int sub = threadIdx.x % kThreadsPerRow;
     const long long nrows = (long long)p.num_tokens * p.num_kv_heads;

@@ -1,0 +1,543 @@
+// Causal (chunked) prefill over the paged 8-bit cache on the 5th-generation
+// tensor cores (tcgen05, accumulators in tensor memory).
+//
+// Source: "1Cat-LLM" README, "Layer 2" (causal online softmax with FP32
+// accumulation, GQA multi-head packing, Wide QK/PV tiles, prefix / causal-tail
+// separation) and "Layer 1" (pages read once and wide); "ReVolta" PyPI page
+// ("Weight and KV formats": 8-bit KV converted to FP16 for compute; chunked
+// prefill with an 8,192-token budget).
+//
+// One CTA owns 128 query rows: 128/G query tokens x the G query heads of one
+// KV head, so every dequantised key/value tile serves all G heads.  Keys come
+// in tiles of 64 (whole cache blocks).  Warp roles (10 warps):
+//   warps 0-3  dequant: E4M3/int8 code tiles -> fp16 K and V tiles, written in
+//              the 128-byte-swizzled canonical layout [d half][key][64 d].
+//              The same bytes are the K-major B operand of S = Q K^T and the
+//              MN-major B operand of O = P V, so V is never transposed.
+//   warps 4-7  softmax: thread i owns row i (TMEM lane i): reads its S row
+//              from TMEM, masks only on tiles that cross the diagonal, keeps
+//              the FP32 running max/sum in registers, writes its fp16 P row
+//              (the A operand of P V) to shared memory, and rescales its O row
+//              in TMEM only when the row maximum grew by more than 2^8.
+//   warp 8     TMA producer: one 2-D tensor copy per cache block and head
+//              into a 3-stage code ring; block ids come from a register window.
+//   warp 9     allocates 256 TMEM columns (S double buffer + O) and issues the
+//              MMAs from one thread: S_j = Q K_j^T overlaps softmax j-1, then
+//              O += P_{j-1} V_{j-1}; completion is signalled with
+//              tcgen05.commit on mbarriers.
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+#include <math.h>
+
+namespace pkvq {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kKT = 64;              // keys per tile
+constexpr int kCodeStages = 3;
+constexpr float kLn2 = 0.693147180559945309f;
+constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
+
+// shared-memory map (offsets from a 1024-byte aligned base)
+constexpr int kOffQ = 0;                                  // 2 halves x [128][128 B]
+constexpr int kOffKV = kOffQ + 32768;                     // 2 bufs x (K 8K+8K, V 8K+8K)
+constexpr int kKVBuf = 32768;
+constexpr int kOffP = kOffKV + 2 * kKVBuf;                // 2 bufs x [128][128 B]
+constexpr int kOffCodes = kOffP + 2 * 16384;              // 3 stages x (K 8K, V 8K)
+constexpr int kCodeStage = 16384;
+constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // 3 x (K 64, V 64) halves
+constexpr int kOffKsf = kOffScl + kCodeStages * 256;            // 2 x 64 fp32 K scales
+constexpr int kOffBars = kOffKsf + 2 * 64 * 4;
+constexpr int kNumBars = 2 + 2 * kCodeStages + 2 * 5;
+constexpr int kOffTaddr = kOffBars + kNumBars * 8;
+constexpr int kSmemBytes = kOffTaddr + 16;
+constexpr size_t kSmemAlloc = kSmemBytes + 1024;
+
+constexpr uint32_t kIdescQK = idesc_f16_f32(128, kKT, false);
+constexpr uint32_t kIdescPV = idesc_f16_f32(128, 128, true);
+
+struct Bars {
+    uint64_t *q_full;
+    uint64_t *code_full, *code_empty;   // [kCodeStages]
+    uint64_t *kv_full, *kv_empty;       // [2]
+    uint64_t *s_full, *s_empty;         // [2]
+    uint64_t *p_full, *pv_done;         // [2]
+    uint64_t *mma_done;                 // all MMAs retired (before TMEM is freed)
+};
+
+__device__ __forceinline__ Bars carve_bars(uint8_t *smem)
+{
+    uint64_t *b = reinterpret_cast<uint64_t *>(smem + kOffBars);
+    Bars r;
+    r.q_full = b;
+    r.code_full = b + 1;
+    r.code_empty = r.code_full + kCodeStages;
+    r.kv_full = r.code_empty + kCodeStages;
+    r.kv_empty = r.kv_full + 2;
+    r.s_full = r.kv_empty + 2;
+    r.s_empty = r.s_full + 2;
+    r.p_full = r.s_empty + 2;
+    r.pv_done = r.p_full + 2;
+    r.mma_done = r.pv_done + 2;
+    return r;
+}
+
+// byte offset of 16-byte chunk c (0..7) of row r in a 128-byte-swizzled tile
+__device__ __forceinline__ uint32_t swz(int r, int c)
+{
+    return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+}
+
+// Every lane waits; the result is made warp-uniform so that a (pathological)
+// timeout makes the whole warp leave its loop together.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, uint32_t *status)
+{
+    const bool ok = mbar_wait(bar, parity, status);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <int KVT>
+__device__ __forceinline__ void cvt4(uint32_t x, uint32_t &lo, uint32_t &hi)
+{
+    if constexpr (KVT == kKvFp8)
+        e4m3x4_to_half2x2(x, lo, hi);
+    else
+        s8x4_to_half2x2(x, lo, hi);
+}
+
+template <int KVT, int BS>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
+                  const __grid_constant__ CUtensorMap vmap, const PrefillParams p)
+{
+    constexpr int kBPT = kKT / BS;   // cache blocks per key tile
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    Bars bars = carve_bars(smem);
+    uint32_t *taddr_smem = reinterpret_cast<uint32_t *>(smem + kOffTaddr);
+
+    const int tile = p.q_tiles - 1 - blockIdx.x;   // longest causal work first
+    const int h = blockIdx.y;
+    const int b = blockIdx.z;
+    const int q_start = p.cu_seqlens_q[b];
+    const int q_len = p.cu_seqlens_q[b + 1] - q_start;
+    const int q0 = tile * p.tokens_per_tile;
+    if (q0 >= q_len || device_wait_failed(p.status))
+        return;
+    const int ctx = p.context_lens[b];
+    const int G = p.group;
+    const int tq_end = min(q_len, q0 + p.tokens_per_tile);
+    const int pos_lo = ctx - q_len + q0;
+    const int pos_hi = ctx - q_len + tq_end - 1;
+    const int nkeys = max(0, min(ctx, pos_hi + 1));
+    const int ntiles = (nkeys + kKT - 1) / kKT;
+    const int nblk_seq = (ctx + BS - 1) / BS;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        mbar_init(bars.q_full, 4);
+        for (int s = 0; s < kCodeStages; ++s) {
+            mbar_init(&bars.code_full[s], 1);
+            mbar_init(&bars.code_empty[s], 4);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars.kv_full[i], 4);
+            mbar_init(&bars.kv_empty[i], 1);
+            mbar_init(&bars.s_full[i], 1);
+            mbar_init(&bars.s_empty[i], 4);
+            mbar_init(&bars.p_full[i], 4);
+            mbar_init(&bars.pv_done[i], 1);
+        }
+        mbar_init(bars.mma_done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(taddr_smem, 256);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *taddr_smem;   // S buffers at +0 / +64, O at +128
+
+    if (warp == 8) {
+        // ------------------------------------------------ TMA producer --
+        if (lane == 0) {
+            prefetch_tmap(&kmap);
+            prefetch_tmap(&vmap);
+        }
+        const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq;
+        const int nblk_used = min(nblk_seq, ntiles * kBPT);
+        int win0 = lane < nblk_used ? __ldg(bt + lane) : 0;
+        int win1 = 32 + lane < nblk_used ? __ldg(bt + 32 + lane) : 0;
+        int wbase = 0;
+        int issued = 0;
+        for (int j = 0; j < ntiles; ++j) {
+            const int s = j % kCodeStages;
+            if (j >= kCodeStages &&
+                !warp_wait(&bars.code_empty[s], ((j - kCodeStages) / kCodeStages) & 1, p.status))
+                break;
+            issued = j + 1;
+            const int blk0 = j * kBPT;
+            const int nb = min(kBPT, nblk_seq - blk0);
+            int ids[kBPT];
+#pragma unroll
+            for (int i = 0; i < kBPT; ++i) {
+                const int bi = blk0 + i;
+                const int a = __shfl_sync(0xffffffffu, win0, bi & 31);
+                const int c = __shfl_sync(0xffffffffu, win1, bi & 31);
+                ids[i] = (bi - wbase) < 32 ? a : c;
+            }
+            if (lane == 0) {
+                uint32_t tx = (uint32_t)nb * BS * 128 * 2;
+                if constexpr (KVT == kKvInt8)
+                    tx += (uint32_t)nb * BS * 2 * 2;
+                mbar_arrive_expect_tx(&bars.code_full[s], tx);
+                uint8_t *dst = smem + kOffCodes + s * kCodeStage;
+                uint16_t *sd = reinterpret_cast<uint16_t *>(smem + kOffScl + s * 256);
+#pragma unroll
+                for (int i = 0; i < kBPT; ++i) {
+                    if (i >= nb)
+                        break;
+                    int phys = ids[i];
+#ifdef PKVQ_BOUNDS_CHECK
+                    if (phys < 0 || phys >= p.num_blocks) {
+                        atomicOr(p.status, kStatusBadBlock);
+                        phys = 0;
+                    }
+#endif
+                    const int y = (phys * p.num_kv_heads + h) * BS;
+                    tma_tile_2d_g2s(dst + i * BS * 128, &kmap, 0, y, &bars.code_full[s]);
+                    tma_tile_2d_g2s(dst + 8192 + i * BS * 128, &vmap, 0, y, &bars.code_full[s]);
+                    if constexpr (KVT == kKvInt8) {
+                        tma_bulk_g2s(sd + i * BS, p.k_scale_tok + (size_t)y, BS * 2,
+                                     &bars.code_full[s]);
+                        tma_bulk_g2s(sd + 64 + i * BS, p.v_scale_tok + (size_t)y, BS * 2,
+                                     &bars.code_full[s]);
+                    }
+                }
+            }
+            if (blk0 + kBPT >= wbase + 32) {
+                wbase += 32;
+                win0 = win1;
+                win1 = wbase + 32 + lane < nblk_used ? __ldg(bt + wbase + 32 + lane) : 0;
+            }
+        }
+        // Copies this CTA issued must land before it exits: wait (bounded) for
+        // the most recent round of every stage (already complete when the
+        // consumers kept up).
+        if (lane == 0)
+            for (int j = max(0, issued - kCodeStages); j < issued; ++j)
+                mbar_wait(&bars.code_full[j % kCodeStages], (j / kCodeStages) & 1, nullptr);
+    } else if (warp == 9) {
+        // --------------------------------------------------- MMA issuer --
+        if (lane == 0 && ntiles > 0) {
+            bool ok = mbar_wait(bars.q_full, 0, p.status);
+            auto pv = [&](int i) -> bool {
+                const int bi = i & 1;
+                if (!mbar_wait(&bars.p_full[bi], (i >> 1) & 1, p.status))
+                    return false;
+                tc_fence_after();
+                const uint32_t pa = sbase + kOffP + bi * 16384;
+                const uint32_t vb = sbase + kOffKV + bi * kKVBuf + 16384;
+#pragma unroll
+                for (int ks = 0; ks < kKT / 16; ++ks) {
+                    const uint64_t ad = desc_sw128(pa + ks * 32, 16, 1024);
+                    const uint64_t bd = desc_sw128(vb + ks * 2048, 8192, 1024);
+                    mma_f16_ss(tmem + 128, ad, bd, kIdescPV, (i > 0 || ks > 0) ? 1u : 0u);
+                }
+                mma_commit(&bars.pv_done[bi]);
+                mma_commit(&bars.kv_empty[bi]);
+                return true;
+            };
+            for (int j = 0; ok && j < ntiles; ++j) {
+                const int bj = j & 1;
+                if (!mbar_wait(&bars.kv_full[bj], (j >> 1) & 1, p.status))
+                    break;
+                if (j >= 2 && !mbar_wait(&bars.s_empty[bj], ((j - 2) >> 1) & 1, p.status))
+                    break;
+                tc_fence_after();
+                const uint32_t qa = sbase + kOffQ;
+                const uint32_t kb = sbase + kOffKV + bj * kKVBuf;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t ad = desc_sw128(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                    const uint64_t bd = desc_sw128(kb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                    mma_f16_ss(tmem + bj * kKT, ad, bd, kIdescQK, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(&bars.s_full[bj]);
+                if (j >= 1 && !pv(j - 1))
+                    ok = false;
+            }
+            if (ok)
+                pv(ntiles - 1);
+            mma_commit(bars.mma_done);
+            mbar_wait(bars.mma_done, 0, p.status);
+        }
+    } else if (warp < 4) {
+        // ------------------------------------------------------ dequant --
+        const int dt = tid;   // 0..127
+        for (int j = 0; j < ntiles; ++j) {
+            const int s = j % kCodeStages, bj = j & 1;
+            if (!warp_wait(&bars.code_full[s], (j / kCodeStages) & 1, p.status))
+                break;
+            if (j >= 2 && !warp_wait(&bars.kv_empty[bj], ((j - 2) >> 1) & 1, p.status))
+                break;
+            const uint8_t *codes = smem + kOffCodes + s * kCodeStage;
+            const uint16_t *scl = reinterpret_cast<const uint16_t *>(smem + kOffScl + s * 256);
+            uint8_t *kv = smem + kOffKV + bj * kKVBuf;
+            const int key0 = j * kKT;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int isv = k >> 2;
+                const int u = dt + 128 * (k & 3);
+                const int row = u & 63, cc = u >> 6;   // key row, 16-byte code chunk
+                const uint4 w = *reinterpret_cast<const uint4 *>(codes + isv * 8192 + swz(row, cc));
+                uint32_t hv[8];
+                cvt4<KVT>(w.x, hv[0], hv[1]);
+                cvt4<KVT>(w.y, hv[2], hv[3]);
+                cvt4<KVT>(w.z, hv[4], hv[5]);
+                cvt4<KVT>(w.w, hv[6], hv[7]);
+                if constexpr (KVT == kKvInt8) {
+                    if (isv) {
+                        const uint32_t sc = scl[64 + row];
+                        const uint32_t s2 = sc | (sc << 16);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            __half2 x = __hmul2(*reinterpret_cast<__half2 *>(&hv[e]),
+                                                *reinterpret_cast<const __half2 *>(&s2));
+                            hv[e] = *reinterpret_cast<uint32_t *>(&x);
+                        }
+                    }
+                }
+                if (key0 + row >= ctx) {   // never-written slot: may hold NaN codes
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        hv[e] = 0u;
+                }
+                uint8_t *dst = kv + isv * 16384 + (cc >> 2) * 8192;
+                *reinterpret_cast<uint4 *>(dst + swz(row, (2 * cc) & 7)) =
+                    make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                *reinterpret_cast<uint4 *>(dst + swz(row, (2 * cc + 1) & 7)) =
+                    make_uint4(hv[4], hv[5], hv[6], hv[7]);
+            }
+            if constexpr (KVT == kKvInt8) {
+                if (dt < 64) {
+                    float *ksf = reinterpret_cast<float *>(smem + kOffKsf) + bj * 64;
+                    ksf[dt] = key0 + dt < ctx ? __half2float(__ushort_as_half(scl[dt])) : 0.0f;
+                }
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars.code_empty[s]);
+                mbar_arrive(&bars.kv_full[bj]);
+            }
+        }
+    } else {
+        // ------------------------------------------------------ softmax --
+        const int r = tid - 128;             // row == TMEM lane
+        const int sw = warp - 4;             // lane quadrant of this warp
+        const uint32_t tl = tmem + ((uint32_t)(32 * sw) << 16);
+        const int tq = q0 + r / G, gq = r % G;
+        const bool valid = r < p.tokens_per_tile * G && tq < q_len;
+        const int pos = ctx - q_len + tq;
+        const size_t qrow = (size_t)(q_start + tq) * p.num_q_heads + (size_t)h * G + gq;
+
+        // Q row -> shared memory (K-major, swizzled), zeros for padding rows
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.q + qrow * kHeadDim);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4 *>(smem + kOffQ + (c >> 3) * 16384 + swz(r, c & 7)) = v;
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bars.q_full);
+        }
+
+        float kfac = p.scale_log2;
+        if constexpr (KVT == kKvFp8)
+            kfac *= __ldg(p.k_scale + h);
+        float m_used = -INFINITY, l = 0.0f;
+        bool ok = true;
+        for (int j = 0; j < ntiles; ++j) {
+            const int bj = j & 1;
+            if (!warp_wait(&bars.s_full[bj], (j >> 1) & 1, p.status)) {
+                ok = false;
+                break;
+            }
+            if constexpr (KVT == kKvInt8) {
+                // the K scales below were written by the dequant warps
+                if (!warp_wait(&bars.kv_full[bj], (j >> 1) & 1, p.status)) {
+                    ok = false;
+                    break;
+                }
+            }
+            tc_fence_after();
+            float sv[kKT];
+            {
+                uint32_t u0[32], u1[32];
+                tmem_ld32(tl + bj * kKT, u0);
+                tmem_ld32(tl + bj * kKT + 32, u1);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    sv[c] = __uint_as_float(u0[c]);
+                    sv[32 + c] = __uint_as_float(u1[c]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&bars.s_empty[bj]);
+
+            const int key0 = j * kKT;
+            const float *ksf = reinterpret_cast<const float *>(smem + kOffKsf) + bj * 64;
+            float mx = -INFINITY;
+            const bool need_mask = key0 + kKT - 1 > pos_lo;
+#pragma unroll
+            for (int c = 0; c < kKT; ++c) {
+                float v = sv[c] * kfac;
+                if constexpr (KVT == kKvInt8)
+                    v *= ksf[c];
+                if (need_mask && key0 + c > pos)
+                    v = -INFINITY;
+                sv[c] = v;
+                mx = fmaxf(mx, v);
+            }
+            // lazy rescale: only when the max grew by more than 2^8
+            const bool need = m_used != -INFINITY && mx > m_used + kRescaleLog2;
+            if (__any_sync(0xffffffffu, need)) {
+                if (!warp_wait(&bars.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float corr = need ? fast_exp2(m_used - mx) : 1.0f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t o[32];
+                    tmem_ld32(tl + 128 + 32 * q, o);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
+                    tmem_st32(tl + 128 + 32 * q, o);
+                }
+                tmem_st_wait();
+                if (need) {
+                    l *= corr;
+                    m_used = mx;
+                }
+            }
+            if (m_used == -INFINITY)
+                m_used = mx;   // first finite max (O is still empty)
+            const float mu = m_used == -INFINITY ? 0.0f : m_used;
+            uint32_t pk[kKT / 2];
+#pragma unroll
+            for (int c = 0; c < kKT; c += 2) {
+                const float p0 = fast_exp2(sv[c] - mu);
+                const float p1 = fast_exp2(sv[c + 1] - mu);
+                l += p0 + p1;
+                pk[c / 2] = pack_half2(p0, p1);
+            }
+            // the P buffer was last read by PV_{j-2}
+            if (j >= 2 && !warp_wait(&bars.pv_done[bj], ((j - 2) >> 1) & 1, p.status)) {
+                ok = false;
+                break;
+            }
+            uint8_t *prow = smem + kOffP + bj * 16384;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4 *>(prow + swz(r, c)) =
+                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&bars.p_full[bj]);
+        }
+
+        // ---- epilogue: O / l -> fp16 ----
+        float vfac = 1.0f;
+        if constexpr (KVT == kKvFp8)
+            vfac = __ldg(p.v_scale + h);
+        const bool have_o = ok && ntiles > 0 &&
+                            warp_wait(&bars.pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1,
+                                      p.status);
+        if (have_o)
+            tc_fence_after();
+        const float f = (have_o && l > 0.0f) ? vfac / l : 0.0f;
+        __half *dst = p.out + qrow * kHeadDim;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t o[32];
+            if (have_o)   // warp-uniform
+                tmem_ld32(tl + 128 + 32 * q, o);
+            if (valid) {
+#pragma unroll
+                for (int c = 0; c < 32; c += 8) {
+                    uint4 w;
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        x[e] = have_o ? __uint_as_float(o[c + e]) * f : 0.0f;
+                    w.x = pack_half2(x[0], x[1]);
+                    w.y = pack_half2(x[2], x[3]);
+                    w.z = pack_half2(x[4], x[5]);
+                    w.w = pack_half2(x[6], x[7]);
+                    *reinterpret_cast<uint4 *>(dst + 32 * q + c) = w;
+                }
+            }
+        }
+        if (valid && p.lse)
+            p.lse[qrow] = (have_o && l > 0.0f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+    }
+
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+template <int KVT, int BS>
+cudaError_t launch_tc(const PrefillParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                      cudaStream_t stream)
+{
+    auto kern = prefill_tc_kernel<KVT, BS>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc);
+    if (e != cudaSuccess)
+        return e;
+    dim3 grid(p.q_tiles, p.num_kv_heads, p.batch);
+    kern<<<grid, kThreads, kSmemAlloc, stream>>>(kmap, vmap, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_tc(const PrefillParams &p, int kv_dtype, const CUtensorMap &kmap,
+                              const CUtensorMap &vmap, cudaStream_t stream)
+{
+    if (p.q_tiles == 0 || p.batch == 0)
+        return cudaSuccess;
+    const bool fp8 = kv_dtype == kKvFp8;
+    switch (p.block_size) {
+    case 16: return fp8 ? launch_tc<kKvFp8, 16>(p, kmap, vmap, stream)
+                        : launch_tc<kKvInt8, 16>(p, kmap, vmap, stream);
+    case 32: return fp8 ? launch_tc<kKvFp8, 32>(p, kmap, vmap, stream)
+                        : launch_tc<kKvInt8, 32>(p, kmap, vmap, stream);
+    case 64: return fp8 ? launch_tc<kKvFp8, 64>(p, kmap, vmap, stream)
+                        : launch_tc<kKvInt8, 64>(p, kmap, vmap, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace pkvq

@@ -1,0 +1,134 @@
+// 5th-generation tensor core (tcgen05) and tensor-memory helpers for sm_100a:
+// TMEM allocation, shared-memory matrix descriptors, single-thread MMA issue
+// with mbarrier commit, and TMEM <-> register moves.  Thin PTX wrappers.
+#pragma once
+
+#include "common.cuh"
+
+namespace pkvq {
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Generic-proxy shared-memory writes become visible to the async proxy
+// (tensor core operand reads).
+__device__ __forceinline__ void fence_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle.  Address, leading and
+// stride byte offsets in bytes (all multiples of 16).  Bits: start >> 4 at
+// [0,14), LBO >> 4 at [16,30), SBO >> 4 at [32,46), descriptor version 1 at
+// [46,48), layout SWIZZLE_128B (2) at [61,64).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor, kind::f16: fp16 A and B, fp32 accumulator, A
+// K-major, B K-major or MN-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major)
+{
+    return (1u << 4)                                  // D format f32
+           | (b_mn_major ? (1u << 16) : 0u)           // B major
+           | ((uint32_t)(N >> 3) << 17)
+           | ((uint32_t)(M >> 4) << 24);
+}
+
+// D[tmem] = A * B (+ D if accumulate), one thread issues.
+__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// The mbarrier gets one arrival when every tcgen05 operation issued so far by
+// this thread has completed.
+__device__ __forceinline__ void mma_commit(uint64_t *bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(bar))
+        : "memory");
+}
+
+#define PKVQ_R32(X)                                                                           \
+    "=r"(X[0]), "=r"(X[1]), "=r"(X[2]), "=r"(X[3]), "=r"(X[4]), "=r"(X[5]), "=r"(X[6]),      \
+        "=r"(X[7]), "=r"(X[8]), "=r"(X[9]), "=r"(X[10]), "=r"(X[11]), "=r"(X[12]),           \
+        "=r"(X[13]), "=r"(X[14]), "=r"(X[15]), "=r"(X[16]), "=r"(X[17]), "=r"(X[18]),        \
+        "=r"(X[19]), "=r"(X[20]), "=r"(X[21]), "=r"(X[22]), "=r"(X[23]), "=r"(X[24]),        \
+        "=r"(X[25]), "=r"(X[26]), "=r"(X[27]), "=r"(X[28]), "=r"(X[29]), "=r"(X[30]),        \
+        "=r"(X[31])
+#define PKVQ_RI32(X)                                                                          \
+    "r"(X[0]), "r"(X[1]), "r"(X[2]), "r"(X[3]), "r"(X[4]), "r"(X[5]), "r"(X[6]), "r"(X[7]),  \
+        "r"(X[8]), "r"(X[9]), "r"(X[10]), "r"(X[11]), "r"(X[12]), "r"(X[13]), "r"(X[14]),    \
+        "r"(X[15]), "r"(X[16]), "r"(X[17]), "r"(X[18]), "r"(X[19]), "r"(X[20]), "r"(X[21]),  \
+        "r"(X[22]), "r"(X[23]), "r"(X[24]), "r"(X[25]), "r"(X[26]), "r"(X[27]), "r"(X[28]),  \
+        "r"(X[29]), "r"(X[30]), "r"(X[31])
+#define PKVQ_LIST32                                                                           \
+    "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,"  \
+    "%24,%25,%26,%27,%28,%29,%30,%31}"
+
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp w reads lanes
+// 32*(w%4) .. +31); the wait is inside, so the registers are ready on return.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 " PKVQ_LIST32 ", [%32];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : PKVQ_R32(r)
+                 : "r"(taddr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,"
+                 "%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+                 PKVQ_RI32(r)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+}  // namespace pkvq
