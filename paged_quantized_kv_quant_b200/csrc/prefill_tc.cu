@@ -7,24 +7,27 @@
 // ("Weight and KV formats": 8-bit KV converted to FP16 for compute; chunked
 // prefill with an 8,192-token budget).
 //
-// One CTA owns 128 query rows: 128/G query tokens x the G query heads of one
-// KV head, so every dequantised key/value tile serves all G heads.  Keys come
-// in tiles of 64 (whole cache blocks).  Warp roles (10 warps):
-//   warps 0-3  dequant: E4M3/int8 code tiles -> fp16 K and V tiles, written in
-//              the 128-byte-swizzled canonical layout [d half][key][64 d].
-//              The same bytes are the K-major B operand of S = Q K^T and the
-//              MN-major B operand of O = P V, so V is never transposed.
-//   warps 4-7  softmax: thread i owns row i (TMEM lane i): reads its S row
-//              from TMEM, masks only on tiles that cross the diagonal, keeps
-//              the FP32 running max/sum in registers, writes its fp16 P row
-//              (the A operand of P V) to shared memory, and rescales its O row
-//              in TMEM only when the row maximum grew by more than 2^8.
-//   warp 8     TMA producer: one 2-D tensor copy per cache block and head
-//              into a 3-stage code ring; block ids come from a register window.
-//   warp 9     allocates 256 TMEM columns (S double buffer + O) and issues the
-//              MMAs from one thread: S_j = Q K_j^T overlaps softmax j-1, then
-//              O += P_{j-1} V_{j-1}; completion is signalled with
-//              tcgen05.commit on mbarriers.
+// A CTA owns two adjacent query tiles A and B of 128 rows each (a tile is
+// 128/G query tokens x the G query heads of one KV head).  Both tiles read the
+// same keys, so every 64-key tile is fetched and dequantised once for 256
+// query rows.  Warp roles (12 warps):
+//   warps 0-1   dequant: E4M3/int8 code tiles -> fp16 K and V tiles in the
+//               128-byte-swizzled canonical layout [d half][key][64 d].  The
+//               same bytes are the K-major B operand of S = Q K^T and the
+//               MN-major B operand of O = P V, so V is never transposed.
+//   warps 4-7   softmax for tile A, warps 8-11 softmax for tile B: thread i of
+//               a group owns row i (TMEM lane i) of its tile: it reads its S
+//               row from TMEM, masks only on tiles that cross the diagonal,
+//               keeps the FP32 running max/sum in registers, writes its fp16 P
+//               row (A operand of P V) to shared memory and rescales its O row
+//               in TMEM only when the row maximum grew by more than 2^8.
+//   warp 2      TMA producer: one 2-D tensor copy per cache block and head
+//               into a 3-stage code ring; block ids come from a register window.
+//   warp 3      allocates all 512 TMEM columns (per tile: S double buffer and
+//               O) and issues every MMA from one thread; the tensor core
+//               alternates between the two tiles, so one group's softmax runs
+//               while the other group's products execute.  Completion is
+//               signalled with tcgen05.commit on mbarriers.
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
@@ -34,26 +37,33 @@
 namespace pkvq {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
 constexpr int kKT = 64;              // keys per tile
 constexpr int kCodeStages = 3;
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
 
+constexpr int kWarpTma = 2;
+constexpr int kWarpMma = 3;
+constexpr int kDequantWarps = 2;
+
 // shared-memory map (offsets from a 1024-byte aligned base)
-constexpr int kOffQ = 0;                                  // 2 halves x [128][128 B]
-constexpr int kOffKV = kOffQ + 32768;                     // 2 bufs x (K 8K+8K, V 8K+8K)
+constexpr int kOffQ = 0;                                  // 2 tiles x 2 halves x [128][128 B]
+constexpr int kQTile = 32768;
+constexpr int kOffKV = kOffQ + 2 * kQTile;                // 2 bufs x (K 8K+8K, V 8K+8K)
 constexpr int kKVBuf = 32768;
-constexpr int kOffP = kOffKV + 2 * kKVBuf;                // 2 bufs x [128][128 B]
-constexpr int kOffCodes = kOffP + 2 * 16384;              // 3 stages x (K 8K, V 8K)
+constexpr int kOffP = kOffKV + 2 * kKVBuf;                // 2 tiles x [128][128 B]
+constexpr int kPTile = 16384;
+constexpr int kOffCodes = kOffP + 2 * kPTile;             // 3 stages x (K 8K, V 8K)
 constexpr int kCodeStage = 16384;
 constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // 3 x (K 64, V 64) halves
-constexpr int kOffKsf = kOffScl + kCodeStages * 256;            // 2 x 64 fp32 K scales
+constexpr int kOffKsf = kOffScl + kCodeStages * 256;            // 2 x 64 fp32 K factors
 constexpr int kOffBars = kOffKsf + 2 * 64 * 4;
-constexpr int kNumBars = 2 + 2 * kCodeStages + 2 * 5;
+constexpr int kNumBars = 1 + 2 * kCodeStages + 2 * 2 + 2 * (2 * 2 + 2) + 1;
 constexpr int kOffTaddr = kOffBars + kNumBars * 8;
 constexpr int kSmemBytes = kOffTaddr + 16;
 constexpr size_t kSmemAlloc = kSmemBytes + 1024;
+static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
 
 constexpr uint32_t kIdescQK = idesc_f16_f32(128, kKT, false);
 constexpr uint32_t kIdescPV = idesc_f16_f32(128, 128, true);
@@ -62,8 +72,8 @@ struct Bars {
     uint64_t *q_full;
     uint64_t *code_full, *code_empty;   // [kCodeStages]
     uint64_t *kv_full, *kv_empty;       // [2]
-    uint64_t *s_full, *s_empty;         // [2]
-    uint64_t *p_full, *pv_done;         // [2]
+    uint64_t *s_full, *s_empty;         // [tile][2]
+    uint64_t *p_full, *pv_done;         // [tile]
     uint64_t *mma_done;                 // all MMAs retired (before TMEM is freed)
 };
 
@@ -77,8 +87,8 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *smem)
     r.kv_full = r.code_empty + kCodeStages;
     r.kv_empty = r.kv_full + 2;
     r.s_full = r.kv_empty + 2;
-    r.s_empty = r.s_full + 2;
-    r.p_full = r.s_empty + 2;
+    r.s_empty = r.s_full + 4;
+    r.p_full = r.s_empty + 4;
     r.pv_done = r.p_full + 2;
     r.mma_done = r.pv_done + 2;
     return r;
@@ -107,6 +117,27 @@ __device__ __forceinline__ void cvt4(uint32_t x, uint32_t &lo, uint32_t &hi)
         s8x4_to_half2x2(x, lo, hi);
 }
 
+// Per-tile geometry of one of the CTA's two query tiles.
+struct QTile {
+    int q0;        // first query token (within the sequence)
+    int pos_lo;    // position of its first token
+    int ntiles;    // key tiles it needs (0: tile absent or sees no key)
+};
+
+__device__ __forceinline__ QTile make_qtile(int tile, int tokens_per_tile, int q_len, int ctx)
+{
+    QTile t;
+    t.q0 = tile * tokens_per_tile;
+    t.pos_lo = ctx - q_len + t.q0;
+    t.ntiles = 0;
+    if (t.q0 < q_len) {
+        const int tq_end = min(q_len, t.q0 + tokens_per_tile);
+        const int nkeys = max(0, min(ctx, ctx - q_len + tq_end));
+        t.ntiles = (nkeys + kKT - 1) / kKT;
+    }
+    return t;
+}
+
 template <int KVT, int BS>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -120,52 +151,52 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     Bars bars = carve_bars(smem);
     uint32_t *taddr_smem = reinterpret_cast<uint32_t *>(smem + kOffTaddr);
 
-    const int tile = p.q_tiles - 1 - blockIdx.x;   // longest causal work first
+    const int npairs = (p.q_tiles + 1) / 2;
+    const int pair = npairs - 1 - blockIdx.x;   // longest causal work first
     const int h = blockIdx.y;
     const int b = blockIdx.z;
     const int q_start = p.cu_seqlens_q[b];
     const int q_len = p.cu_seqlens_q[b + 1] - q_start;
-    const int q0 = tile * p.tokens_per_tile;
-    if (q0 >= q_len || device_wait_failed(p.status))
+    if (2 * pair * p.tokens_per_tile >= q_len || device_wait_failed(p.status))
         return;
     const int ctx = p.context_lens[b];
     const int G = p.group;
-    const int tq_end = min(q_len, q0 + p.tokens_per_tile);
-    const int pos_lo = ctx - q_len + q0;
-    const int pos_hi = ctx - q_len + tq_end - 1;
-    const int nkeys = max(0, min(ctx, pos_hi + 1));
-    const int ntiles = (nkeys + kKT - 1) / kKT;
+    const QTile qt[2] = {make_qtile(2 * pair, p.tokens_per_tile, q_len, ctx),
+                         make_qtile(2 * pair + 1, p.tokens_per_tile, q_len, ctx)};
+    const int ntiles = max(qt[0].ntiles, qt[1].ntiles);
     const int nblk_seq = (ctx + BS - 1) / BS;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
-        mbar_init(bars.q_full, 4);
+        mbar_init(bars.q_full, 8);
         for (int s = 0; s < kCodeStages; ++s) {
             mbar_init(&bars.code_full[s], 1);
-            mbar_init(&bars.code_empty[s], 4);
+            mbar_init(&bars.code_empty[s], kDequantWarps);
         }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars.kv_full[i], 4);
+            mbar_init(&bars.kv_full[i], kDequantWarps);
             mbar_init(&bars.kv_empty[i], 1);
-            mbar_init(&bars.s_full[i], 1);
-            mbar_init(&bars.s_empty[i], 4);
             mbar_init(&bars.p_full[i], 4);
             mbar_init(&bars.pv_done[i], 1);
+        }
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&bars.s_full[i], 1);
+            mbar_init(&bars.s_empty[i], 4);
         }
         mbar_init(bars.mma_done, 1);
         fence_mbar_init();
     }
-    if (warp == 9) {
-        tmem_alloc(taddr_smem, 256);
+    if (warp == kWarpMma) {
+        tmem_alloc(taddr_smem, 512);
         tmem_relinquish();
         tc_fence_before();
     }
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *taddr_smem;   // S buffers at +0 / +64, O at +128
+    const uint32_t tmem = *taddr_smem;   // tile x: S buffers at x*256 + {0, 64}, O at x*256 + 128
 
-    if (warp == 8) {
+    if (warp == kWarpTma) {
         // ------------------------------------------------ TMA producer --
         if (lane == 0) {
             prefetch_tmap(&kmap);
@@ -234,54 +265,73 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         if (lane == 0)
             for (int j = max(0, issued - kCodeStages); j < issued; ++j)
                 mbar_wait(&bars.code_full[j % kCodeStages], (j / kCodeStages) & 1, nullptr);
-    } else if (warp == 9) {
+    } else if (warp == kWarpMma) {
         // --------------------------------------------------- MMA issuer --
         if (lane == 0 && ntiles > 0) {
             bool ok = mbar_wait(bars.q_full, 0, p.status);
-            auto pv = [&](int i) -> bool {
-                const int bi = i & 1;
-                if (!mbar_wait(&bars.p_full[bi], (i >> 1) & 1, p.status))
+            auto pv = [&](int x, int i) -> bool {   // O_x += P_x(i) V(i)
+                if (!mbar_wait(&bars.p_full[x], i & 1, p.status))
                     return false;
                 tc_fence_after();
-                const uint32_t pa = sbase + kOffP + bi * 16384;
-                const uint32_t vb = sbase + kOffKV + bi * kKVBuf + 16384;
+                const uint32_t pa = sbase + kOffP + x * kPTile;
+                const uint32_t vb = sbase + kOffKV + (i & 1) * kKVBuf + 16384;
 #pragma unroll
                 for (int ks = 0; ks < kKT / 16; ++ks) {
                     const uint64_t ad = desc_sw128(pa + ks * 32, 16, 1024);
                     const uint64_t bd = desc_sw128(vb + ks * 2048, 8192, 1024);
-                    mma_f16_ss(tmem + 128, ad, bd, kIdescPV, (i > 0 || ks > 0) ? 1u : 0u);
+                    mma_f16_ss(tmem + x * 256 + 128, ad, bd, kIdescPV,
+                               (i > 0 || ks > 0) ? 1u : 0u);
                 }
-                mma_commit(&bars.pv_done[bi]);
-                mma_commit(&bars.kv_empty[bi]);
+                mma_commit(&bars.pv_done[x]);
                 return true;
             };
             for (int j = 0; ok && j < ntiles; ++j) {
                 const int bj = j & 1;
                 if (!mbar_wait(&bars.kv_full[bj], (j >> 1) & 1, p.status))
                     break;
-                if (j >= 2 && !mbar_wait(&bars.s_empty[bj], ((j - 2) >> 1) & 1, p.status))
-                    break;
-                tc_fence_after();
-                const uint32_t qa = sbase + kOffQ;
                 const uint32_t kb = sbase + kOffKV + bj * kKVBuf;
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t ad = desc_sw128(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                    const uint64_t bd = desc_sw128(kb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-                    mma_f16_ss(tmem + bj * kKT, ad, bd, kIdescQK, ks > 0 ? 1u : 0u);
+                for (int x = 0; x < 2; ++x) {
+                    if (j >= qt[x].ntiles)
+                        continue;
+                    if (j >= 2 &&
+                        !mbar_wait(&bars.s_empty[x * 2 + bj], ((j - 2) >> 1) & 1, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t qa = sbase + kOffQ + x * kQTile;
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint64_t ad =
+                            desc_sw128(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                        const uint64_t bd =
+                            desc_sw128(kb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                        mma_f16_ss(tmem + x * 256 + bj * kKT, ad, bd, kIdescQK, ks > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&bars.s_full[x * 2 + bj]);
                 }
-                mma_commit(&bars.s_full[bj]);
-                if (j >= 1 && !pv(j - 1))
-                    ok = false;
+                if (!ok)
+                    break;
+                if (j >= 1) {
+#pragma unroll
+                    for (int x = 0; x < 2; ++x)
+                        if (j - 1 < qt[x].ntiles && !pv(x, j - 1))
+                            ok = false;
+                    mma_commit(&bars.kv_empty[(j - 1) & 1]);
+                }
             }
             if (ok)
-                pv(ntiles - 1);
+                for (int x = 0; x < 2; ++x)
+                    if (qt[x].ntiles == ntiles)
+                        pv(x, ntiles - 1);
             mma_commit(bars.mma_done);
             mbar_wait(bars.mma_done, 0, p.status);
         }
-    } else if (warp < 4) {
+    } else if (warp < kDequantWarps) {
         // ------------------------------------------------------ dequant --
-        const int dt = tid;   // 0..127
+        const int row = tid;   // 0..63: this thread converts key row `row` of K and V
+        const float kfac = p.scale_log2;
         for (int j = 0; j < ntiles; ++j) {
             const int s = j % kCodeStages, bj = j & 1;
             if (!warp_wait(&bars.code_full[s], (j / kCodeStages) & 1, p.status))
@@ -292,11 +342,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             const uint16_t *scl = reinterpret_cast<const uint16_t *>(smem + kOffScl + s * 256);
             uint8_t *kv = smem + kOffKV + bj * kKVBuf;
             const int key0 = j * kKT;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int isv = k >> 2;
-                const int u = dt + 128 * (k & 3);
-                const int row = u & 63, cc = u >> 6;   // key row, 16-byte code chunk
+#pragma unroll 4
+            for (int k = 0; k < 16; ++k) {
+                const int isv = k >> 3;
+                const int cc = k & 7;   // 16-byte code chunk
                 const uint4 w = *reinterpret_cast<const uint4 *>(codes + isv * 8192 + swz(row, cc));
                 uint32_t hv[8];
                 cvt4<KVT>(w.x, hv[0], hv[1]);
@@ -327,10 +376,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     make_uint4(hv[4], hv[5], hv[6], hv[7]);
             }
             if constexpr (KVT == kKvInt8) {
-                if (dt < 64) {
-                    float *ksf = reinterpret_cast<float *>(smem + kOffKsf) + bj * 64;
-                    ksf[dt] = key0 + dt < ctx ? __half2float(__ushort_as_half(scl[dt])) : 0.0f;
-                }
+                // per-key score factor: softmax scale * log2(e) * K scale
+                float *ksf = reinterpret_cast<float *>(smem + kOffKsf) + bj * 64;
+                ksf[row] =
+                    key0 + row < ctx ? kfac * __half2float(__ushort_as_half(scl[row])) : 0.0f;
             }
             fence_async_smem();
             __syncwarp();
@@ -339,23 +388,26 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 mbar_arrive(&bars.kv_full[bj]);
             }
         }
-    } else {
+    } else if (warp >= 4) {
         // ------------------------------------------------------ softmax --
-        const int r = tid - 128;             // row == TMEM lane
-        const int sw = warp - 4;             // lane quadrant of this warp
-        const uint32_t tl = tmem + ((uint32_t)(32 * sw) << 16);
-        const int tq = q0 + r / G, gq = r % G;
-        const bool valid = r < p.tokens_per_tile * G && tq < q_len;
+        const int x = (warp - 4) >> 2;       // query tile of this group
+        const int r = tid - 128 - 128 * x;   // row == TMEM lane
+        const int sw = warp & 3;             // lane quadrant of this warp
+        const uint32_t tl = tmem + ((uint32_t)(32 * sw) << 16) + x * 256;
+        const QTile T = qt[x];
+        const int tq = T.q0 + r / G, gq = r % G;
+        const bool valid = r < p.tokens_per_tile * G && tq < q_len;   // rows that exist
         const int pos = ctx - q_len + tq;
         const size_t qrow = (size_t)(q_start + tq) * p.num_q_heads + (size_t)h * G + gq;
 
         // Q row -> shared memory (K-major, swizzled), zeros for padding rows
         {
             const uint4 *src = reinterpret_cast<const uint4 *>(p.q + qrow * kHeadDim);
+            uint8_t *qs = smem + kOffQ + x * kQTile;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-                *reinterpret_cast<uint4 *>(smem + kOffQ + (c >> 3) * 16384 + swz(r, c & 7)) = v;
+                *reinterpret_cast<uint4 *>(qs + (c >> 3) * 16384 + swz(r, c & 7)) = v;
             }
             fence_async_smem();
             __syncwarp();
@@ -368,54 +420,74 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             kfac *= __ldg(p.k_scale + h);
         float m_used = -INFINITY, l = 0.0f;
         bool ok = true;
-        for (int j = 0; j < ntiles; ++j) {
+        for (int j = 0; j < T.ntiles; ++j) {
             const int bj = j & 1;
-            if (!warp_wait(&bars.s_full[bj], (j >> 1) & 1, p.status)) {
+            if (!warp_wait(&bars.s_full[x * 2 + bj], (j >> 1) & 1, p.status)) {
                 ok = false;
                 break;
             }
             if constexpr (KVT == kKvInt8) {
-                // the K scales below were written by the dequant warps
+                // the per-key factors below were written by the dequant warps
                 if (!warp_wait(&bars.kv_full[bj], (j >> 1) & 1, p.status)) {
                     ok = false;
                     break;
                 }
             }
             tc_fence_after();
-            float sv[kKT];
+            float v[kKT];
             {
-                uint32_t u0[32], u1[32];
-                tmem_ld32(tl + bj * kKT, u0);
-                tmem_ld32(tl + bj * kKT + 32, u1);
+                uint32_t ua[32], ub[32];
+                tmem_ld64(tl + bj * kKT, ua, ub);
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
-                    sv[c] = __uint_as_float(u0[c]);
-                    sv[32 + c] = __uint_as_float(u1[c]);
+                    v[c] = __uint_as_float(ua[c]);
+                    v[32 + c] = __uint_as_float(ub[c]);
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&bars.s_empty[bj]);
+                mbar_arrive(&bars.s_empty[x * 2 + bj]);
 
             const int key0 = j * kKT;
-            const float *ksf = reinterpret_cast<const float *>(smem + kOffKsf) + bj * 64;
-            float mx = -INFINITY;
-            const bool need_mask = key0 + kKT - 1 > pos_lo;
+            if constexpr (KVT == kKvFp8) {
+                const float2 f2 = make_float2(kfac, kfac);
 #pragma unroll
-            for (int c = 0; c < kKT; ++c) {
-                float v = sv[c] * kfac;
-                if constexpr (KVT == kKvInt8)
-                    v *= ksf[c];
-                if (need_mask && key0 + c > pos)
-                    v = -INFINITY;
-                sv[c] = v;
-                mx = fmaxf(mx, v);
+                for (int c = 0; c < kKT; c += 2) {
+                    const float2 r2 = __fmul2_rn(make_float2(v[c], v[c + 1]), f2);
+                    v[c] = r2.x, v[c + 1] = r2.y;
+                }
+            } else {
+                const float *ksf = reinterpret_cast<const float *>(smem + kOffKsf) + bj * 64;
+#pragma unroll
+                for (int c = 0; c < kKT; c += 2) {
+                    const float2 r2 = __fmul2_rn(make_float2(v[c], v[c + 1]),
+                                                 make_float2(ksf[c], ksf[c + 1]));
+                    v[c] = r2.x, v[c + 1] = r2.y;
+                }
             }
-            // lazy rescale: only when the max grew by more than 2^8
+            if (key0 + kKT - 1 > T.pos_lo) {   // a key may lie past a row's position
+#pragma unroll
+                for (int c = 0; c < kKT; ++c)
+                    if (key0 + c > pos)
+                        v[c] = -INFINITY;
+            }
+            // row max: eight independent chains, then a tree
+            float m8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                m8[i] = v[i];
+#pragma unroll
+                for (int c = i + 8; c < kKT; c += 8)
+                    m8[i] = fmaxf(m8[i], v[c]);
+            }
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            // lazy rescale: only when the max grew by more than 2^8 (this needs
+            // the previous P V product to have landed in O)
             const bool need = m_used != -INFINITY && mx > m_used + kRescaleLog2;
             if (__any_sync(0xffffffffu, need)) {
-                if (!warp_wait(&bars.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.status)) {
+                if (!warp_wait(&bars.pv_done[x], (j - 1) & 1, p.status)) {
                     ok = false;
                     break;
                 }
@@ -439,20 +511,26 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             if (m_used == -INFINITY)
                 m_used = mx;   // first finite max (O is still empty)
             const float mu = m_used == -INFINITY ? 0.0f : m_used;
+            const float2 nmu = make_float2(-mu, -mu);
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
             uint32_t pk[kKT / 2];
 #pragma unroll
             for (int c = 0; c < kKT; c += 2) {
-                const float p0 = fast_exp2(sv[c] - mu);
-                const float p1 = fast_exp2(sv[c + 1] - mu);
-                l += p0 + p1;
-                pk[c / 2] = pack_half2(p0, p1);
+                const float2 d = __fadd2_rn(make_float2(v[c], v[c + 1]), nmu);
+                const float2 e = make_float2(fast_exp2(d.x), fast_exp2(d.y));
+                acc[(c >> 1) & 3] = __fadd2_rn(acc[(c >> 1) & 3], e);
+                pk[c / 2] = pack_half2(e.x, e.y);
             }
-            // the P buffer was last read by PV_{j-2}
-            if (j >= 2 && !warp_wait(&bars.pv_done[bj], ((j - 2) >> 1) & 1, p.status)) {
+            const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+            const float2 a = __fadd2_rn(a01, a23);
+            l += a.x + a.y;
+            // the P buffer was last read by P V of the previous tile
+            if (j >= 1 && !warp_wait(&bars.pv_done[x], (j - 1) & 1, p.status)) {
                 ok = false;
                 break;
             }
-            uint8_t *prow = smem + kOffP + bj * 16384;
+            uint8_t *prow = smem + kOffP + x * kPTile;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
                 *reinterpret_cast<uint4 *>(prow + swz(r, c)) =
@@ -461,16 +539,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&bars.p_full[bj]);
+                mbar_arrive(&bars.p_full[x]);
         }
 
         // ---- epilogue: O / l -> fp16 ----
         float vfac = 1.0f;
         if constexpr (KVT == kKvFp8)
             vfac = __ldg(p.v_scale + h);
-        const bool have_o = ok && ntiles > 0 &&
-                            warp_wait(&bars.pv_done[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1,
-                                      p.status);
+        const bool have_o = ok && T.ntiles > 0 &&
+                            warp_wait(&bars.pv_done[x], (T.ntiles - 1) & 1, p.status);
         if (have_o)
             tc_fence_after();
         const float f = (have_o && l > 0.0f) ? vfac / l : 0.0f;
@@ -483,15 +560,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             if (valid) {
 #pragma unroll
                 for (int c = 0; c < 32; c += 8) {
-                    uint4 w;
-                    float x[8];
+                    float y[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        x[e] = have_o ? __uint_as_float(o[c + e]) * f : 0.0f;
-                    w.x = pack_half2(x[0], x[1]);
-                    w.y = pack_half2(x[2], x[3]);
-                    w.z = pack_half2(x[4], x[5]);
-                    w.w = pack_half2(x[6], x[7]);
+                        y[e] = have_o ? __uint_as_float(o[c + e]) * f : 0.0f;
+                    uint4 w;
+                    w.x = pack_half2(y[0], y[1]);
+                    w.y = pack_half2(y[2], y[3]);
+                    w.z = pack_half2(y[4], y[5]);
+                    w.w = pack_half2(y[6], y[7]);
                     *reinterpret_cast<uint4 *>(dst + 32 * q + c) = w;
                 }
             }
@@ -501,9 +578,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     }
 
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kWarpMma) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -516,7 +593,7 @@ cudaError_t launch_tc(const PrefillParams &p, const CUtensorMap &kmap, const CUt
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc);
     if (e != cudaSuccess)
         return e;
-    dim3 grid(p.q_tiles, p.num_kv_heads, p.batch);
+    dim3 grid((p.q_tiles + 1) / 2, p.num_kv_heads, p.batch);
     kern<<<grid, kThreads, kSmemAlloc, stream>>>(kmap, vmap, p);
     return cudaGetLastError();
 }
