@@ -22,7 +22,7 @@
 //               row (A operand of P V) to shared memory and rescales its O row
 //               in TMEM only when the row maximum grew by more than 2^8.
 //   warp 2      TMA producer: one 2-D tensor copy per cache block and head
-//               into a 3-stage code ring; block ids come from a register window.
+//               into a 2-stage code ring; block ids come from a register window.
 //   warp 3      allocates all 512 TMEM columns (per tile: S double buffer and
 //               O) and issues every MMA from one thread; the tensor core
 //               alternates between the two tiles, so one group's softmax runs
@@ -39,7 +39,8 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kKT = 64;              // keys per tile
-constexpr int kCodeStages = 3;
+constexpr int kCodeStages = 2;
+constexpr int kKVBufs = 3;         // dequantised K/V tiles in flight
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
 
@@ -50,16 +51,16 @@ constexpr int kDequantWarps = 2;
 // shared-memory map (offsets from a 1024-byte aligned base)
 constexpr int kOffQ = 0;                                  // 2 tiles x 2 halves x [128][128 B]
 constexpr int kQTile = 32768;
-constexpr int kOffKV = kOffQ + 2 * kQTile;                // 2 bufs x (K 8K+8K, V 8K+8K)
+constexpr int kOffKV = kOffQ + 2 * kQTile;                // 3 bufs x (K 8K+8K, V 8K+8K)
 constexpr int kKVBuf = 32768;
-constexpr int kOffP = kOffKV + 2 * kKVBuf;                // 2 tiles x [128][128 B]
+constexpr int kOffP = kOffKV + kKVBufs * kKVBuf;          // 2 tiles x [128][128 B]
 constexpr int kPTile = 16384;
-constexpr int kOffCodes = kOffP + 2 * kPTile;             // 3 stages x (K 8K, V 8K)
+constexpr int kOffCodes = kOffP + 2 * kPTile;             // 2 stages x (K 8K, V 8K)
 constexpr int kCodeStage = 16384;
-constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // 3 x (K 64, V 64) halves
-constexpr int kOffKsf = kOffScl + kCodeStages * 256;            // 2 x 64 fp32 K factors
-constexpr int kOffBars = kOffKsf + 2 * 64 * 4;
-constexpr int kNumBars = 1 + 2 * kCodeStages + 2 * 2 + 2 * (2 * 2 + 2) + 1;
+constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // stages x (K 64, V 64) halves
+constexpr int kOffKsf = kOffScl + kCodeStages * 256;            // bufs x 64 fp32 K factors
+constexpr int kOffBars = kOffKsf + kKVBufs * 64 * 4;
+constexpr int kNumBars = 1 + 2 * kCodeStages + 2 * kKVBufs + 2 * (2 * 2 + 2) + 1;
 constexpr int kOffTaddr = kOffBars + kNumBars * 8;
 constexpr int kSmemBytes = kOffTaddr + 16;
 constexpr size_t kSmemAlloc = kSmemBytes + 1024;
@@ -71,7 +72,7 @@ constexpr uint32_t kIdescPV = idesc_f16_f32(128, 128, true);
 struct Bars {
     uint64_t *q_full;
     uint64_t *code_full, *code_empty;   // [kCodeStages]
-    uint64_t *kv_full, *kv_empty;       // [2]
+    uint64_t *kv_full, *kv_empty;       // [kKVBufs]
     uint64_t *s_full, *s_empty;         // [tile][2]
     uint64_t *p_full, *pv_done;         // [tile]
     uint64_t *mma_done;                 // all MMAs retired (before TMEM is freed)
@@ -85,8 +86,8 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *smem)
     r.code_full = b + 1;
     r.code_empty = r.code_full + kCodeStages;
     r.kv_full = r.code_empty + kCodeStages;
-    r.kv_empty = r.kv_full + 2;
-    r.s_full = r.kv_empty + 2;
+    r.kv_empty = r.kv_full + kKVBufs;
+    r.s_full = r.kv_empty + kKVBufs;
     r.s_empty = r.s_full + 4;
     r.p_full = r.s_empty + 4;
     r.pv_done = r.p_full + 2;
@@ -174,9 +175,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             mbar_init(&bars.code_full[s], 1);
             mbar_init(&bars.code_empty[s], kDequantWarps);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kKVBufs; ++i) {
             mbar_init(&bars.kv_full[i], kDequantWarps);
             mbar_init(&bars.kv_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&bars.p_full[i], 4);
             mbar_init(&bars.pv_done[i], 1);
         }
@@ -274,7 +277,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     return false;
                 tc_fence_after();
                 const uint32_t pa = sbase + kOffP + x * kPTile;
-                const uint32_t vb = sbase + kOffKV + (i & 1) * kKVBuf + 16384;
+                const uint32_t vb = sbase + kOffKV + (i % kKVBufs) * kKVBuf + 16384;
 #pragma unroll
                 for (int ks = 0; ks < kKT / 16; ++ks) {
                     const uint64_t ad = desc_sw128(pa + ks * 32, 16, 1024);
@@ -286,10 +289,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 return true;
             };
             for (int j = 0; ok && j < ntiles; ++j) {
-                const int bj = j & 1;
-                if (!mbar_wait(&bars.kv_full[bj], (j >> 1) & 1, p.status))
+                const int bj = j & 1;            // S buffer
+                const int kvb = j % kKVBufs;     // K/V buffer
+                if (!mbar_wait(&bars.kv_full[kvb], (j / kKVBufs) & 1, p.status))
                     break;
-                const uint32_t kb = sbase + kOffKV + bj * kKVBuf;
+                const uint32_t kb = sbase + kOffKV + kvb * kKVBuf;
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     if (j >= qt[x].ntiles)
@@ -318,7 +322,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     for (int x = 0; x < 2; ++x)
                         if (j - 1 < qt[x].ntiles && !pv(x, j - 1))
                             ok = false;
-                    mma_commit(&bars.kv_empty[(j - 1) & 1]);
+                    mma_commit(&bars.kv_empty[(j - 1) % kKVBufs]);
                 }
             }
             if (ok)
@@ -333,10 +337,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         const int row = tid;   // 0..63: this thread converts key row `row` of K and V
         const float kfac = p.scale_log2;
         for (int j = 0; j < ntiles; ++j) {
-            const int s = j % kCodeStages, bj = j & 1;
+            const int s = j % kCodeStages, bj = j % kKVBufs;
             if (!warp_wait(&bars.code_full[s], (j / kCodeStages) & 1, p.status))
                 break;
-            if (j >= 2 && !warp_wait(&bars.kv_empty[bj], ((j - 2) >> 1) & 1, p.status))
+            if (j >= kKVBufs &&
+                !warp_wait(&bars.kv_empty[bj], ((j - kKVBufs) / kKVBufs) & 1, p.status))
                 break;
             const uint8_t *codes = smem + kOffCodes + s * kCodeStage;
             const uint16_t *scl = reinterpret_cast<const uint16_t *>(smem + kOffScl + s * 256);
@@ -428,7 +433,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             }
             if constexpr (KVT == kKvInt8) {
                 // the per-key factors below were written by the dequant warps
-                if (!warp_wait(&bars.kv_full[bj], (j >> 1) & 1, p.status)) {
+                if (!warp_wait(&bars.kv_full[j % kKVBufs], (j / kKVBufs) & 1, p.status)) {
                     ok = false;
                     break;
                 }
@@ -458,7 +463,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     v[c] = r2.x, v[c + 1] = r2.y;
                 }
             } else {
-                const float *ksf = reinterpret_cast<const float *>(smem + kOffKsf) + bj * 64;
+                const float *ksf =
+                    reinterpret_cast<const float *>(smem + kOffKsf) + (j % kKVBufs) * 64;
 #pragma unroll
                 for (int c = 0; c < kKT; c += 2) {
                     const float2 r2 = __fmul2_rn(make_float2(v[c], v[c + 1]),
