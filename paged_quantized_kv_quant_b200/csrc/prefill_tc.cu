@@ -10,24 +10,27 @@
 // A CTA owns two adjacent query tiles A and B of 128 rows each (a tile is
 // 128/G query tokens x the G query heads of one KV head).  Both tiles read the
 // same keys, so every 64-key tile is fetched and dequantised once for 256
-// query rows.  Warp roles (12 warps):
+// query rows.  Q and P are kept in tensor memory, so the MMAs read only the
+// fp16 K/V tiles from shared memory (operand bandwidth, not arithmetic, is
+// what bounds a 128 x 64 product).  Warp roles (12 warps):
 //   warps 0-1   dequant: E4M3/int8 code tiles -> fp16 K and V tiles in the
 //               128-byte-swizzled canonical layout [d half][key][64 d].  The
 //               same bytes are the K-major B operand of S = Q K^T and the
 //               MN-major B operand of O = P V, so V is never transposed.
-//   warps 4-7   softmax for tile A, warps 8-11 softmax for tile B: thread i of
-//               a group owns row i (TMEM lane i) of its tile: it reads its S
-//               row from TMEM, masks only on tiles that cross the diagonal,
-//               keeps the FP32 running max/sum in registers, writes its fp16 P
-//               row (A operand of P V) to shared memory and rescales its O row
-//               in TMEM only when the row maximum grew by more than 2^8.
 //   warp 2      TMA producer: one 2-D tensor copy per cache block and head
-//               into a 2-stage code ring; block ids come from a register window.
-//   warp 3      allocates all 512 TMEM columns (per tile: S double buffer and
-//               O) and issues every MMA from one thread; the tensor core
-//               alternates between the two tiles, so one group's softmax runs
-//               while the other group's products execute.  Completion is
-//               signalled with tcgen05.commit on mbarriers.
+//               into a 3-stage code ring; block ids come from a register window.
+//   warp 3      allocates all 512 TMEM columns (per tile: S/P 64, O 128, Q 64)
+//               and issues every MMA from one thread, ping-ponging between the
+//               tiles: O_A += P_A V, S_A = Q_A K_next, then the same for B.
+//               Completion is signalled with tcgen05.commit on mbarriers.
+//   warps 4-7   softmax for tile A, warps 8-11 softmax for tile B: thread i of
+//               a group owns row i (TMEM lane i): it stores its Q row in TMEM,
+//               reads its S row, masks only on tiles that cross the diagonal,
+//               keeps the FP32 running max/sum in registers, writes its fp16 P
+//               row over the S columns it came from, and rescales its O row in
+//               TMEM only when the row maximum grew by more than 2^8.  The
+//               tensor core runs one group's products while the other group's
+//               softmax runs.
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
@@ -39,8 +42,8 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kKT = 64;              // keys per tile
-constexpr int kCodeStages = 2;
-constexpr int kKVBufs = 3;         // dequantised K/V tiles in flight
+constexpr int kCodeStages = 3;
+constexpr int kKVBufs = 4;           // dequantised K/V tiles in flight
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
 
@@ -48,19 +51,18 @@ constexpr int kWarpTma = 2;
 constexpr int kWarpMma = 3;
 constexpr int kDequantWarps = 2;
 
+// tensor memory, per query tile x at x * 256: S/P (P in the first 32), O, Q
+constexpr uint32_t kTmS = 0, kTmO = 64, kTmQ = 192;
+
 // shared-memory map (offsets from a 1024-byte aligned base)
-constexpr int kOffQ = 0;                                  // 2 tiles x 2 halves x [128][128 B]
-constexpr int kQTile = 32768;
-constexpr int kOffKV = kOffQ + 2 * kQTile;                // 3 bufs x (K 8K+8K, V 8K+8K)
+constexpr int kOffKV = 0;                                 // bufs x (K 8K+8K, V 8K+8K)
 constexpr int kKVBuf = 32768;
-constexpr int kOffP = kOffKV + kKVBufs * kKVBuf;          // 2 tiles x [128][128 B]
-constexpr int kPTile = 16384;
-constexpr int kOffCodes = kOffP + 2 * kPTile;             // 2 stages x (K 8K, V 8K)
+constexpr int kOffCodes = kOffKV + kKVBufs * kKVBuf;      // stages x (K 8K, V 8K)
 constexpr int kCodeStage = 16384;
 constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // stages x (K 64, V 64) halves
 constexpr int kOffKsf = kOffScl + kCodeStages * 256;            // bufs x 64 fp32 K factors
 constexpr int kOffBars = kOffKsf + kKVBufs * 64 * 4;
-constexpr int kNumBars = 1 + 2 * kCodeStages + 2 * kKVBufs + 2 * (2 * 2 + 2) + 1;
+constexpr int kNumBars = 1 + 2 * kCodeStages + 2 * kKVBufs + 3 * 2 + 1;
 constexpr int kOffTaddr = kOffBars + kNumBars * 8;
 constexpr int kSmemBytes = kOffTaddr + 16;
 constexpr size_t kSmemAlloc = kSmemBytes + 1024;
@@ -73,8 +75,7 @@ struct Bars {
     uint64_t *q_full;
     uint64_t *code_full, *code_empty;   // [kCodeStages]
     uint64_t *kv_full, *kv_empty;       // [kKVBufs]
-    uint64_t *s_full, *s_empty;         // [tile][2]
-    uint64_t *p_full, *pv_done;         // [tile]
+    uint64_t *s_full, *p_full, *pv_done;   // [tile]
     uint64_t *mma_done;                 // all MMAs retired (before TMEM is freed)
 };
 
@@ -88,8 +89,7 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *smem)
     r.kv_full = r.code_empty + kCodeStages;
     r.kv_empty = r.kv_full + kKVBufs;
     r.s_full = r.kv_empty + kKVBufs;
-    r.s_empty = r.s_full + 4;
-    r.p_full = r.s_empty + 4;
+    r.p_full = r.s_full + 2;
     r.pv_done = r.p_full + 2;
     r.mma_done = r.pv_done + 2;
     return r;
@@ -180,12 +180,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             mbar_init(&bars.kv_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars.s_full[i], 1);
             mbar_init(&bars.p_full[i], 4);
             mbar_init(&bars.pv_done[i], 1);
-        }
-        for (int i = 0; i < 4; ++i) {
-            mbar_init(&bars.s_full[i], 1);
-            mbar_init(&bars.s_empty[i], 4);
         }
         mbar_init(bars.mma_done, 1);
         fence_mbar_init();
@@ -197,7 +194,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     }
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *taddr_smem;   // tile x: S buffers at x*256 + {0, 64}, O at x*256 + 128
+    const uint32_t tmem = *taddr_smem;
 
     if (warp == kWarpTma) {
         // ------------------------------------------------ TMA producer --
@@ -272,63 +269,52 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         // --------------------------------------------------- MMA issuer --
         if (lane == 0 && ntiles > 0) {
             bool ok = mbar_wait(bars.q_full, 0, p.status);
-            auto pv = [&](int x, int i) -> bool {   // O_x += P_x(i) V(i)
-                if (!mbar_wait(&bars.p_full[x], i & 1, p.status))
+            tc_fence_after();
+            auto qk = [&](int x, int j) -> bool {   // S_x = Q_x K(j)^T
+                const int kvb = j % kKVBufs;
+                if (!mbar_wait(&bars.kv_full[kvb], (j / kKVBufs) & 1, p.status))
                     return false;
                 tc_fence_after();
-                const uint32_t pa = sbase + kOffP + x * kPTile;
-                const uint32_t vb = sbase + kOffKV + (i % kKVBufs) * kKVBuf + 16384;
+                const uint32_t kb = sbase + kOffKV + kvb * kKVBuf;
+                const uint32_t tx = tmem + x * 256;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t bd = desc_sw128(kb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+                    mma_f16_ts(tx + kTmS, tx + kTmQ + ks * 8, bd, kIdescQK, ks > 0 ? 1u : 0u);
+                }
+                mma_commit(&bars.s_full[x]);
+                return true;
+            };
+            auto pv = [&](int x, int j) -> bool {   // O_x += P_x(j) V(j)
+                if (!mbar_wait(&bars.p_full[x], j & 1, p.status))
+                    return false;
+                tc_fence_after();
+                const uint32_t vb = sbase + kOffKV + (j % kKVBufs) * kKVBuf + 16384;
+                const uint32_t tx = tmem + x * 256;
 #pragma unroll
                 for (int ks = 0; ks < kKT / 16; ++ks) {
-                    const uint64_t ad = desc_sw128(pa + ks * 32, 16, 1024);
                     const uint64_t bd = desc_sw128(vb + ks * 2048, 8192, 1024);
-                    mma_f16_ss(tmem + x * 256 + 128, ad, bd, kIdescPV,
-                               (i > 0 || ks > 0) ? 1u : 0u);
+                    mma_f16_ts(tx + kTmO, tx + kTmS + ks * 8, bd, kIdescPV,
+                               (j > 0 || ks > 0) ? 1u : 0u);
                 }
                 mma_commit(&bars.pv_done[x]);
                 return true;
             };
+            for (int x = 0; ok && x < 2; ++x)
+                if (qt[x].ntiles > 0 && !qk(x, 0))
+                    ok = false;
             for (int j = 0; ok && j < ntiles; ++j) {
-                const int bj = j & 1;            // S buffer
-                const int kvb = j % kKVBufs;     // K/V buffer
-                if (!mbar_wait(&bars.kv_full[kvb], (j / kKVBufs) & 1, p.status))
-                    break;
-                const uint32_t kb = sbase + kOffKV + kvb * kKVBuf;
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    if (j >= qt[x].ntiles)
+                    if (!ok || j >= qt[x].ntiles)
                         continue;
-                    if (j >= 2 &&
-                        !mbar_wait(&bars.s_empty[x * 2 + bj], ((j - 2) >> 1) & 1, p.status)) {
+                    // The next S overwrites this tile's P in the same columns;
+                    // the tensor core executes a thread's MMAs in issue order.
+                    if (!pv(x, j) || (j + 1 < qt[x].ntiles && !qk(x, j + 1)))
                         ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t qa = sbase + kOffQ + x * kQTile;
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint64_t ad =
-                            desc_sw128(qa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                        const uint64_t bd =
-                            desc_sw128(kb + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
-                        mma_f16_ss(tmem + x * 256 + bj * kKT, ad, bd, kIdescQK, ks > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&bars.s_full[x * 2 + bj]);
                 }
-                if (!ok)
-                    break;
-                if (j >= 1) {
-#pragma unroll
-                    for (int x = 0; x < 2; ++x)
-                        if (j - 1 < qt[x].ntiles && !pv(x, j - 1))
-                            ok = false;
-                    mma_commit(&bars.kv_empty[(j - 1) % kKVBufs]);
-                }
+                mma_commit(&bars.kv_empty[j % kKVBufs]);
             }
-            if (ok)
-                for (int x = 0; x < 2; ++x)
-                    if (qt[x].ntiles == ntiles)
-                        pv(x, ntiles - 1);
             mma_commit(bars.mma_done);
             mbar_wait(bars.mma_done, 0, p.status);
         }
@@ -405,16 +391,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         const int pos = ctx - q_len + tq;
         const size_t qrow = (size_t)(q_start + tq) * p.num_q_heads + (size_t)h * G + gq;
 
-        // Q row -> shared memory (K-major, swizzled), zeros for padding rows
+        // Q row -> tensor memory (two fp16 per column), zeros for padding rows
         {
             const uint4 *src = reinterpret_cast<const uint4 *>(p.q + qrow * kHeadDim);
-            uint8_t *qs = smem + kOffQ + x * kQTile;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-                *reinterpret_cast<uint4 *>(qs + (c >> 3) * 16384 + swz(r, c & 7)) = v;
+            for (int half = 0; half < 2; ++half) {
+                uint32_t w[32];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 v = valid ? __ldg(src + half * 8 + c) : make_uint4(0u, 0u, 0u, 0u);
+                    w[4 * c] = v.x, w[4 * c + 1] = v.y, w[4 * c + 2] = v.z, w[4 * c + 3] = v.w;
+                }
+                tmem_st32(tl + kTmQ + 32 * half, w);
             }
-            fence_async_smem();
+            tmem_st_wait();
+            tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(bars.q_full);
@@ -426,8 +417,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         float m_used = -INFINITY, l = 0.0f;
         bool ok = true;
         for (int j = 0; j < T.ntiles; ++j) {
-            const int bj = j & 1;
-            if (!warp_wait(&bars.s_full[x * 2 + bj], (j >> 1) & 1, p.status)) {
+            // S(j) complete also means P V of tile j-1 has completed (in-order MMAs)
+            if (!warp_wait(&bars.s_full[x], j & 1, p.status)) {
                 ok = false;
                 break;
             }
@@ -442,17 +433,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             float v[kKT];
             {
                 uint32_t ua[32], ub[32];
-                tmem_ld64(tl + bj * kKT, ua, ub);
+                tmem_ld64(tl + kTmS, ua, ub);
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
                     v[c] = __uint_as_float(ua[c]);
                     v[32 + c] = __uint_as_float(ub[c]);
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&bars.s_empty[x * 2 + bj]);
 
             const int key0 = j * kKT;
             if constexpr (KVT == kKvFp8) {
@@ -489,26 +476,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             }
             const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                    fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-            // lazy rescale: only when the max grew by more than 2^8 (this needs
-            // the previous P V product to have landed in O)
+            // lazy rescale: only when the max grew by more than 2^8
             const bool need = m_used != -INFINITY && mx > m_used + kRescaleLog2;
             if (__any_sync(0xffffffffu, need)) {
-                if (!warp_wait(&bars.pv_done[x], (j - 1) & 1, p.status)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
                 const float corr = need ? fast_exp2(m_used - mx) : 1.0f;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     uint32_t o[32];
-                    tmem_ld32(tl + 128 + 32 * q, o);
+                    tmem_ld32(tl + kTmO + 32 * q, o);
 #pragma unroll
                     for (int c = 0; c < 32; ++c)
                         o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
-                    tmem_st32(tl + 128 + 32 * q, o);
+                    tmem_st32(tl + kTmO + 32 * q, o);
                 }
-                tmem_st_wait();
                 if (need) {
                     l *= corr;
                     m_used = mx;
@@ -531,17 +511,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
             const float2 a = __fadd2_rn(a01, a23);
             l += a.x + a.y;
-            // the P buffer was last read by P V of the previous tile
-            if (j >= 1 && !warp_wait(&bars.pv_done[x], (j - 1) & 1, p.status)) {
-                ok = false;
-                break;
-            }
-            uint8_t *prow = smem + kOffP + x * kPTile;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4 *>(prow + swz(r, c)) =
-                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            fence_async_smem();
+            // P row over the first 32 S columns (the A operand of P V)
+            tmem_st32(tl + kTmS, pk);
+            tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -562,7 +534,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         for (int q = 0; q < 4; ++q) {
             uint32_t o[32];
             if (have_o)   // warp-uniform
-                tmem_ld32(tl + 128 + 32 * q, o);
+                tmem_ld32(tl + kTmO + 32 * q, o);
             if (valid) {
 #pragma unroll
                 for (int c = 0; c < 32; c += 8) {
