@@ -199,6 +199,13 @@ PKVQ_API const char *pkvq_status_string(pkvq_status status);
  */
 PKVQ_API pkvq_status pkvq_device_status(uint32_t *status_out, int32_t clear);
 
+/*
+ * Text of the last CUDA runtime failure seen by this thread inside the library
+ * (the call that failed and cudaGetErrorString of its code), or "" if none.
+ * The pointer stays valid until this thread's next library call.
+ */
+PKVQ_API const char *pkvq_last_error(void);
+
 /* Library version as "major.minor.patch". */
 PKVQ_API const char *pkvq_version(void);
 

@@ -36,12 +36,16 @@ EXPORTED = (
     "pkvq_status_string",
     "pkvq_device_status",
     "pkvq_version",
+    "pkvq_last_error",
 )
 
 
 class PkvqError(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        detail = ""
+        if status == 6:
+            detail = ": " + _lib().pkvq_last_error().decode()
+        super().__init__(f"{what}: {status_string(status)} (status {status}){detail}")
         self.status = status
 
 
@@ -94,6 +98,8 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pkvq_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), I32]
     lib.pkvq_version.restype = ctypes.c_char_p
     lib.pkvq_version.argtypes = []
+    lib.pkvq_last_error.restype = ctypes.c_char_p
+    lib.pkvq_last_error.argtypes = []
     _libs[path] = lib
     return lib
 

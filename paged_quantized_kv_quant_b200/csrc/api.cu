@@ -9,6 +9,7 @@
 #include <cudaTypedefs.h>
 #include <math.h>
 #include <mutex>
+#include <stdio.h>
 #include <stdlib.h>
 
 namespace pkvq {
@@ -94,9 +95,15 @@ pkvq_status cache_maps(const pkvq_cache *c, CUtensorMap *km, CUtensorMap *vm)
     return PKVQ_OK;
 }
 
-pkvq_status from_cuda(cudaError_t e)
+thread_local char t_last_error[256] = "";
+
+pkvq_status from_cuda(cudaError_t e, const char *what = "launch")
 {
-    return e == cudaSuccess ? PKVQ_OK : PKVQ_ERR_CUDA;
+    if (e == cudaSuccess)
+        return PKVQ_OK;
+    snprintf(t_last_error, sizeof(t_last_error), "%s: %s (%d)", what, cudaGetErrorString(e),
+             (int)e);
+    return PKVQ_ERR_CUDA;
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -138,6 +145,11 @@ int device_sm_count()
 using namespace pkvq;
 
 extern "C" {
+
+const char *pkvq_last_error(void)
+{
+    return t_last_error;
+}
 
 const char *pkvq_version(void)
 {
