@@ -11,6 +11,11 @@ GPU) divided by the step time.  Causal prefill TFLOP/s (8,192-token prefill,
 same heads) is reported beside it under "secondary".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pkvq|reference]
+    python bench.py --only decode|prefill [--steps K] [--warmup W]
+
+--only runs nothing but W + K calls of one kernel path on its workload (the
+decode call on the batch-8 x 32K cache, or the 8K causal prefill) and prints
+their average time: the command the ncu captures are taken with.
 
 Under torchrun every rank runs the same batch on its own GPU (no collective on
 the data path: weak scaling); the time is the max over ranks.  The reference
@@ -60,6 +65,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--only", choices=["decode", "prefill"], default=None)
     return ap.parse_args()
 
 
@@ -268,8 +274,84 @@ def time_graph(graph, reps, stream, barrier=None):
     return e0.elapsed_time(e1) / reps
 
 
+DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_b8_ctx32k_fp8_ncu.md")
+DECODE_SOURCES = ("paged_quantized_kv_quant_b200/csrc/decode.cu",
+                  "paged_quantized_kv_quant_b200/csrc/common.cuh")
+
+
+def decode_sources_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def decode_traffic_from_profile():
+    """DRAM bytes (read + write) of one decode call, split and merge kernels,
+    from the committed ncu summary; None when the summary is missing or was
+    taken on other decode sources than the ones built now."""
+    import re
+    try:
+        with open(DECODE_PROFILE) as f:
+            text = f.read()
+    except OSError:
+        return None
+    m = re.search(r"dram_bytes_per_call:\s*([0-9]+)", text)
+    d = re.search(r"decode_sources_digest:\s*([0-9a-f]+)", text)
+    if not m or not d or d.group(1) != decode_sources_digest():
+        return None
+    return int(m.group(1))
+
+
+def run_only(args):
+    """W + K calls of one path, nothing else (for profiler captures)."""
+    import paged_quantized_kv_quant_b200 as pk
+    pk.load_library()
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    stream = torch.cuda.Stream(device=device)
+    if args.only == "decode":
+        spec = synth.workload(DECODE_WORKLOAD)
+        case = synth.make_case(spec)
+        caches, inp, max_ctx, _ = build_decode(case, device)
+        calls = [lambda c=c: decode_step(pk, c, inp, max_ctx, case.softmax_scale, write=False)
+                 for c in caches]
+    else:
+        spec = synth.workload(PREFILL_WORKLOAD)
+        case = synth.make_case(spec)
+        c = pk.PagedKVCache.allocate(spec.kv_dtype, case.num_blocks, spec.block_size,
+                                     spec.num_kv_heads, device=device,
+                                     k_scale=case.k_scale, v_scale=case.v_scale)
+        pk.kv_write_quant(c, case.k.to(device), case.v.to(device), case.slot_mapping.to(device))
+        q = case.q.to(device)
+        out = torch.empty_like(q)
+        cu, bt, ctx = (case.cu_seqlens_q.to(device), case.block_table.to(device),
+                       case.context_lens.to(device))
+        mq = max(spec.q_lens)
+        calls = [lambda: pk.paged_attn_prefill(c, q, cu, bt, ctx, mq, case.softmax_scale,
+                                               out=out)]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(max(0, args.warmup)):
+            calls[i % len(calls)]()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(max(1, args.steps)):
+            calls[i % len(calls)]()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    print(json.dumps({"only": args.only, "workload": spec.name, "calls": max(1, args.steps),
+                      "ms_per_call": e0.elapsed_time(e1) / max(1, args.steps)}), flush=True)
+
+
 def main():
     args = parse()
+    if args.only:
+        run_only(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -421,14 +503,7 @@ def main():
                          f"{nb} KV bytes), FP64 oracle, {dt:.1f} s"}
 
     launches_per_step = 2 + (1 if plan_splits else 0)
-    traffic = None
-    tr_path = os.path.join(ROOT, "profiles", "decode_b8_ctx32k_traffic.json")
-    if os.path.exists(tr_path):
-        try:
-            with open(tr_path) as f:
-                traffic = json.load(f).get("dram_bytes_per_launch")
-        except Exception:
-            traffic = None
+    traffic = decode_traffic_from_profile()
     line = {
         "metric": METRIC,
         "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": 2 * warm,

@@ -225,7 +225,7 @@ size_t pkvq_decode_workspace_bytes(int32_t batch, int32_t q_len, int32_t num_q_h
         max_context_len < 0 || num_q_heads <= 0 || num_q_heads % cache->num_kv_heads)
         return 0;
     DecodePlan plan;
-    if (!decode_plan(batch, q_len, num_q_heads, cache->num_kv_heads, cache->block_size,
+    if (!decode_plan(cache->dtype, batch, q_len, num_q_heads, cache->num_kv_heads, cache->block_size,
                      max_context_len, &plan))
         return 0;
     return plan.workspace_bytes;
@@ -260,7 +260,7 @@ pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void *q, void 
     if ((long long)max_blocks_per_seq * cache->block_size < max_context_len)
         return PKVQ_ERR_INVALID_ARG;
     DecodePlan plan;
-    if (!decode_plan(batch, q_len, num_q_heads, cache->num_kv_heads, cache->block_size,
+    if (!decode_plan(cache->dtype, batch, q_len, num_q_heads, cache->num_kv_heads, cache->block_size,
                      max_context_len, &plan))
         return PKVQ_ERR_INVALID_ARG;
     if (plan.workspace_bytes > 0) {

@@ -500,10 +500,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     float vfac = 1.0f;
     if constexpr (KVT == kKvFp8)
         vfac = __ldg(p.v_scale + h);
+    // Rows are independent: the loop is unrolled so that their shared-memory
+    // reads and global stores overlap.
+#pragma unroll 4
     for (int r = 0; r < RC; ++r) {
         const int rr = rg * RC + r;
         if (rr >= p.rows)
-            break;
+            continue;
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w)
@@ -526,18 +529,22 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
             const size_t wrow =
                 (((size_t)b * p.num_kv_heads + h) * p.num_splits + split) * p.rows + rr;
             p.ws_o[wrow * kHeadDim + d] = O;
-            if (d == 0) {
-                p.ws_ml[wrow * 2] = M;
-                p.ws_ml[wrow * 2 + 1] = L;
-            }
+            if (d == 0)
+                *reinterpret_cast<float2 *>(p.ws_ml + wrow * 2) = make_float2(M, L);
         }
     }
 }
 
 // Merge of the split partial states (one warp per output row):
 // M = max_i m_i, L = sum_i l_i 2^(m_i - M), O = sum_i O_i 2^(m_i - M) / L.
-// Lane i reads split i's (m, l); the O rows are then read four splits at a
-// time so their loads overlap.
+// The splits are taken kMergeChunk at a time: every lane issues the loads of
+// a whole chunk (the (m, l) pairs, the same for all lanes, and its float4 of
+// each O row) before using any, so a chunk costs one memory round trip; the
+// chunks are combined online.  The first chunk is loaded without waiting for
+// the context length (splits past the last one that holds keys are loaded
+// from the workspace but not used).
+constexpr int kMergeChunk = 16;
+
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -553,51 +560,45 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
     const int nblk = (ctx + p.block_size - 1) / p.block_size;
     const int nvalid = min(p.num_splits, (nblk + p.blocks_per_split - 1) / p.blocks_per_split);
     const size_t base = ((size_t)b * p.num_kv_heads + h) * p.num_splits * p.rows + rr;
-    float M = -INFINITY;
-    for (int s = lane; s < nvalid; s += 32)
-        M = fmaxf(M, p.ws_ml[(base + (size_t)s * p.rows) * 2]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float Mu = M == -INFINITY ? 0.0f : M;
-    float L = 0.0f;
+    float M = -INFINITY, L = 0.0f;
     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < nvalid; s0 += 32) {
-        // weights of splits s0 .. s0+31, one per lane
-        const int sl = s0 + lane;
-        float e = 0.0f;
-        if (sl < nvalid) {
-            const size_t wrow = base + (size_t)sl * p.rows;
-            e = fast_exp2(p.ws_ml[wrow * 2] - Mu);
-            L += p.ws_ml[wrow * 2 + 1] * e;
-        }
-        const int n = min(32, nvalid - s0);
-        int j = 0;
-        for (; j + 4 <= n; j += 4) {
-            float4 v[4];
-            float w[4];
+    for (int s0 = 0; s0 < p.num_splits; s0 += kMergeChunk) {
+        if (s0 > 0 && s0 >= nvalid)
+            break;
+        float2 ml[kMergeChunk];
+        float4 v[kMergeChunk];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                w[k] = __shfl_sync(0xffffffffu, e, j + k);
-                v[k] = reinterpret_cast<const float4 *>(
-                    p.ws_o + (base + (size_t)(s0 + j + k) * p.rows) * kHeadDim)[lane];
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                O.x += v[k].x * w[k], O.y += v[k].y * w[k];
-                O.z += v[k].z * w[k], O.w += v[k].w * w[k];
+        for (int k = 0; k < kMergeChunk; ++k) {
+            ml[k] = make_float2(-INFINITY, 0.0f);
+            v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (s0 + k < p.num_splits) {
+                const size_t wrow = base + (size_t)(s0 + k) * p.rows;
+                ml[k] = *reinterpret_cast<const float2 *>(p.ws_ml + wrow * 2);
+                v[k] = reinterpret_cast<const float4 *>(p.ws_o + wrow * kHeadDim)[lane];
             }
         }
-        for (; j < n; ++j) {
-            const float w = __shfl_sync(0xffffffffu, e, j);
-            const float4 v = reinterpret_cast<const float4 *>(
-                p.ws_o + (base + (size_t)(s0 + j) * p.rows) * kHeadDim)[lane];
-            O.x += v.x * w, O.y += v.y * w, O.z += v.z * w, O.w += v.w * w;
+#pragma unroll
+        for (int k = 0; k < kMergeChunk; ++k)
+            if (s0 + k >= nvalid) {
+                ml[k] = make_float2(-INFINITY, 0.0f);
+                v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        float cm = M;
+#pragma unroll
+        for (int k = 0; k < kMergeChunk; ++k)
+            cm = fmaxf(cm, ml[k].x);
+        const float mu = cm == -INFINITY ? 0.0f : cm;
+        const float corr = fast_exp2(M - mu);
+        L *= corr;
+        O.x *= corr, O.y *= corr, O.z *= corr, O.w *= corr;
+#pragma unroll
+        for (int k = 0; k < kMergeChunk; ++k) {
+            const float e = fast_exp2(ml[k].x - mu);
+            L += ml[k].y * e;
+            O.x += v[k].x * e, O.y += v[k].y * e, O.z += v[k].z * e, O.w += v[k].w * e;
         }
+        M = cm;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        L += __shfl_xor_sync(0xffffffffu, L, o);
     const float vfac = p.v_scale ? __ldg(p.v_scale + h) : 1.0f;
     const int tq = rr / p.group, gq = rr % p.group;
     const size_t orow = ((size_t)b * p.q_len + tq) * p.num_q_heads + h * p.group + gq;
@@ -645,10 +646,56 @@ cudaError_t launch_bs(const DecodeParams &p, const CUtensorMap &kmap, const CUte
     }
 }
 
+template <int KVT, int NT, int BS>
+int occupancy_of()
+{
+    auto kern = decode_split_kernel<KVT, NT, BS>;
+    constexpr size_t smem = decode_smem_bytes<BS>();
+    int n = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, smem) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+template <int KVT, int NT>
+int occupancy_bs(int block_size)
+{
+    switch (block_size) {
+    case 16: return occupancy_of<KVT, NT, 16>();
+    case 32: return occupancy_of<KVT, NT, 32>();
+    case 64: return occupancy_of<KVT, NT, 64>();
+    default: return 0;
+    }
+}
+
+// Resident split CTAs per SM for one kernel instance (registers and shared
+// memory decide it), cached per device; 2 where it cannot be queried.
+int split_occupancy(int kv_dtype, int nt, int block_size)
+{
+    constexpr int kMaxDev = 64;
+    static int cache[kMaxDev][2][2][3] = {};
+    int dev = 0;
+    const int bi = block_size == 16 ? 0 : (block_size == 32 ? 1 : 2);
+    const int di = kv_dtype == kKvFp8 ? 0 : 1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+        return 2;
+    int &c = cache[dev][di][nt - 1][bi];
+    if (!c) {
+        int n = di == 0 ? (nt == 1 ? occupancy_bs<kKvFp8, 1>(block_size)
+                                   : occupancy_bs<kKvFp8, 2>(block_size))
+                        : (nt == 1 ? occupancy_bs<kKvInt8, 1>(block_size)
+                                   : occupancy_bs<kKvInt8, 2>(block_size));
+        c = n > 0 ? n : 2;
+    }
+    return c;
+}
+
 }  // namespace
 
-bool decode_plan(int batch, int q_len, int num_q_heads, int num_kv_heads, int block_size,
-                 int max_context_len, DecodePlan *plan)
+bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv_heads,
+                 int block_size, int max_context_len, DecodePlan *plan)
 {
     if (batch <= 0 || q_len <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads)
         return false;
@@ -659,17 +706,26 @@ bool decode_plan(int batch, int q_len, int num_q_heads, int num_kv_heads, int bl
     plan->row_groups = (rows + plan->rows_per_cta - 1) / plan->rows_per_cta;
     const int max_blocks = (max_context_len + block_size - 1) / block_size;
     const long long units = (long long)batch * num_kv_heads * plan->row_groups;
-    // Aim for about `ctas_per_sm` resident CTAs on every SM in a single wave;
-    // never split below one block per warp.
-    int ctas_per_sm = 2;
+    // At most `ctas_per_sm` CTAs on every SM (3, or what fits), all resident
+    // in one wave, with the same number of blocks each: rounding the split
+    // count up instead would put one more CTA on some SMs, and those SMs'
+    // CTAs would all finish last (a memory-bound CTA gets a share of its
+    // SM's bandwidth).  More resident CTAs keep more copies in flight.  Never
+    // split below kMinBlocksPerWarp blocks per warp: short splits pay the
+    // fixed start-up and merge costs for little streaming.
+    // PKVQ_DECODE_CTAS_PER_SM (1..16) replaces the target as given, even
+    // beyond what fits in one wave.
+    constexpr int kMinBlocksPerWarp = 3;
+    int ctas_per_sm = min(3, split_occupancy(kv_dtype, plan->nt, block_size));
     if (const char *env = getenv("PKVQ_DECODE_CTAS_PER_SM")) {
         const int v = atoi(env);
         if (v >= 1 && v <= 16)
             ctas_per_sm = v;
     }
     const long long target = (long long)ctas_per_sm * device_sm_count();
-    long long splits = (target + units - 1) / units;
-    const long long max_splits = max(1, (max_blocks + kWarps - 1) / kWarps);
+    long long splits = target / units;
+    const long long max_splits =
+        max(1, max_blocks / (kWarps * kMinBlocksPerWarp));
     splits = max(1LL, min(splits, max_splits));
     int bps = max_blocks > 0 ? (int)((max_blocks + splits - 1) / splits) : 1;
     splits = max_blocks > 0 ? (max_blocks + bps - 1) / bps : 1;

@@ -53,9 +53,10 @@ struct DecodePlan {
     size_t workspace_bytes;
 };
 
-// Split plan for a decode shape on the current device.
-bool decode_plan(int batch, int q_len, int num_q_heads, int num_kv_heads, int block_size,
-                 int max_context_len, DecodePlan *plan);
+// Split plan for a decode shape on the current device (kv_dtype: kKvFp8 or
+// kKvInt8, whose kernels differ in registers and so in occupancy).
+bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv_heads,
+                 int block_size, int max_context_len, DecodePlan *plan);
 
 cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_dtype,
                           const CUtensorMap &kmap, const CUtensorMap &vmap,

@@ -72,14 +72,14 @@ def test_noalloc_decode_matches_workspace_decode_twice(order):
 def test_noalloc_rejects_shapes_beyond_its_scratch(monkeypatch):
     # a split plan with many CTAs per SM needs more than the fixed 8 MiB
     monkeypatch.setenv("PKVQ_DECODE_CTAS_PER_SM", "16")
-    spec = synth.CaseSpec("decode", synth.FP8_E4M3, 64, 4, [4096] * 4, [2] * 4, seed=42)
+    spec = synth.CaseSpec("decode", synth.FP8_E4M3, 64, 4, [16384] * 4, [2] * 4, seed=42)
     case = synth.make_case(spec)
     cache = gpu_cache(case)
     q = case.q.view(4, 2, 64, 128).cuda()
-    need = pk.decode_workspace_bytes(cache, 4, 2, 64, 4096)
+    need = pk.decode_workspace_bytes(cache, 4, 2, 64, 16384)
     assert need > (8 << 20)
     out = torch.empty_like(q)
     lse = torch.empty((4, 2, 64), dtype=torch.float32, device="cuda")
-    rc = _noalloc(cache, q, case.block_table.cuda(), case.context_lens.cuda(), 4096,
+    rc = _noalloc(cache, q, case.block_table.cuda(), case.context_lens.cuda(), 16384,
                   case.softmax_scale, out, lse)
     assert rc == 4   # PKVQ_ERR_WORKSPACE_TOO_SMALL, nothing launched
