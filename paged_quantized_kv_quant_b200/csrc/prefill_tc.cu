@@ -269,26 +269,29 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         // --------------------------------------------------- MMA issuer --
         // Serves whichever query tile has its P ready (no head-of-line
         // blocking between the two softmax groups); a K/V buffer is released
-        // once every tile that uses it has issued its P V product.
-        if (lane == 0 && ntiles > 0) {
-            bool ok = mbar_wait(bars.q_full, 0, p.status);
+        // once every tile that uses it has issued its P V product.  The whole
+        // warp runs this loop on warp-uniform values (every wait and probe is
+        // made uniform by a vote) and one elected lane issues each tcgen05
+        // instruction.
+        if (ntiles > 0) {
+            bool ok = warp_wait(bars.q_full, 0, p.status);
             tc_fence_after();
             // descriptors of K/V buffer 0; buffer b adds b * kKVBuf bytes
             const uint64_t kd0 = desc_sw128(sbase + kOffKV, 16, 1024);
             const uint64_t vd0 = desc_sw128(sbase + kOffKV + 16384, 8192, 1024);
             auto qk = [&](int x, int j) -> bool {   // S_x = Q_x K(j)^T
                 const int kvb = j % kKVBufs;
-                if (!mbar_wait(&bars.kv_full[kvb], (j / kKVBufs) & 1, p.status))
+                if (!warp_wait(&bars.kv_full[kvb], (j / kKVBufs) & 1, p.status))
                     return false;
                 tc_fence_after();
                 const uint32_t tx = tmem + x * 256;
                 const uint64_t kd = kd0 + (uint64_t)((kvb * kKVBuf) >> 4);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_f16_ts(tx + kTmS, tx + kTmQ + ks * 8,
-                               kd + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4), kIdescQK,
-                               ks > 0 ? 1u : 0u);
-                mma_commit(&bars.s_full[x]);
+                    mma_f16_ts_elect(tx + kTmS, tx + kTmQ + ks * 8,
+                                     kd + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4),
+                                     kIdescQK, ks > 0 ? 1u : 0u);
+                mma_commit_elect(&bars.s_full[x]);
                 return true;
             };
             auto pv = [&](int x, int j) {   // O_x += P_x(j) V(j); P_x(j) is ready
@@ -297,22 +300,28 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 const uint64_t vd = vd0 + (uint64_t)(((j % kKVBufs) * kKVBuf) >> 4);
 #pragma unroll
                 for (int ks = 0; ks < kKT / 16; ++ks)
-                    mma_f16_ts(tx + kTmO, tx + kTmS + ks * 8, vd + (uint64_t)((ks * 2048) >> 4),
-                               kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
-                mma_commit(&bars.pv_done[x]);
+                    mma_f16_ts_elect(tx + kTmO, tx + kTmS + ks * 8,
+                                     vd + (uint64_t)((ks * 2048) >> 4), kIdescPV,
+                                     (j > 0 || ks > 0) ? 1u : 0u);
+                mma_commit_elect(&bars.pv_done[x]);
             };
             for (int x = 0; ok && x < 2; ++x)
                 if (qt[x].ntiles > 0 && !qk(x, 0))
                     ok = false;
             int nxt[2] = {0, 0};   // next P V tile of each query tile
             int released = 0;      // K/V tiles released so far
-            uint64_t t_last = global_timer_ns();
+            // Both tiles are polled with the non-blocking test_wait: a
+            // suspending try_wait on one tile's barrier would leave the other
+            // tile's ready P unserved.  The clock is read every 256 idle polls.
+            uint64_t t_last = 0;
+            uint32_t idle = 0;
             while (ok && (nxt[0] < qt[0].ntiles || nxt[1] < qt[1].ntiles)) {
                 bool progressed = false;
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     const int j = nxt[x];
-                    if (j >= qt[x].ntiles || !mbar_try_wait(&bars.p_full[x], j & 1))
+                    if (j >= qt[x].ntiles ||
+                        !__any_sync(0xffffffffu, mbar_test_wait(&bars.p_full[x], j & 1)))
                         continue;
                     pv(x, j);
                     nxt[x] = j + 1;
@@ -326,18 +335,25 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 }
                 while (released < ntiles && (released >= qt[0].ntiles || nxt[0] > released) &&
                        (released >= qt[1].ntiles || nxt[1] > released)) {
-                    mma_commit(&bars.kv_empty[released % kKVBufs]);
+                    mma_commit_elect(&bars.kv_empty[released % kKVBufs]);
                     ++released;
                 }
                 if (progressed) {
-                    t_last = global_timer_ns();
-                } else if (global_timer_ns() - t_last > kWaitLimitNs) {
-                    atomicOr(p.status, kStatusWaitTimeout);
-                    ok = false;
+                    idle = 0;
+                } else if ((++idle & 255u) == 0) {
+                    // lane 0's clock decides, so that the warp stays converged
+                    const uint64_t now = __shfl_sync(0xffffffffu, global_timer_ns(), 0);
+                    if (idle == 256u) {
+                        t_last = now;   // first check of this idle stretch
+                    } else if (now - t_last > kWaitLimitNs) {
+                        if (lane == 0)
+                            atomicOr(p.status, kStatusWaitTimeout);
+                        ok = false;
+                    }
                 }
             }
-            mma_commit(bars.mma_done);
-            mbar_wait(bars.mma_done, 0, p.status);
+            mma_commit_elect(bars.mma_done);
+            warp_wait(bars.mma_done, 0, p.status);
         }
     } else if (warp < kDequantWarps) {
         // ------------------------------------------------------ dequant --
