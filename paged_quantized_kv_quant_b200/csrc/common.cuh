@@ -77,6 +77,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// Wait for a phase for at most about `ns` nanoseconds, suspended (the thread
+// takes no issue slots while it sleeps and wakes as soon as the phase
+// completes); returns whether the phase completed.
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t *bar, uint32_t parity, uint32_t ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Non-blocking probe of a phase (test_wait never suspends the thread, unlike
 // try_wait): for a thread that polls several barriers in turn.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
