@@ -52,6 +52,8 @@ def decode_config(spec, world: int):
             "l2": "inputs larger than L2: two 268 MB caches alternated step by step",
             "parallelism": f"dp{world} (independent batches per GPU)"}
 PREFILL_WORKLOAD = 3
+REFERENCE_BUDGET_S = 120.0
+E2E_GRAPH_STEPS = 8
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -158,43 +160,66 @@ def _oracle_cache(case):
     return oc
 
 
-def oracle_decode_sample(case, n_seqs: int):
-    """Times the FP64 oracle on all heads of the first n_seqs sequences of the
-    decode batch; returns (KV bytes of those sequences, seconds, threads)."""
+def _oracle_rows(oc, case, rows):
+    """One oracle pass over the given (sequence, query head) rows; seconds, threads."""
     import oracle
-    oc = _oracle_cache(case)
-    s = case.spec
-    rows = np.array([[b, h] for b in range(n_seqs) for h in range(s.num_q_heads)], np.int32)
     t0 = time.perf_counter()
     _, _, used = oracle.paged_attention(oc, _bits16(case.q), case.cu_seqlens_q.numpy(),
                                         case.context_lens.numpy(), case.block_table.numpy(),
-                                        case.softmax_scale, rows=rows)
-    dt = time.perf_counter() - t0
-    per_seq = synth.kv_read_bytes(s) // len(s.context_lens)
-    return per_seq * n_seqs, dt, used, oc
+                                        case.softmax_scale,
+                                        rows=np.asarray(rows, np.int32).reshape(-1, 2))
+    return time.perf_counter() - t0, used
+
+
+def _row_bytes(spec) -> float:
+    """Algorithmic KV bytes per (sequence, query head) row: a 1/Hq share of
+    its sequence's KV bytes (the G rows of a KV head read the same codes)."""
+    return synth.kv_read_bytes(spec) / len(spec.context_lens) / spec.num_q_heads
+
+
+def oracle_decode_sample(case, min_seconds: float = 10.0, max_passes: int = 4):
+    """Times the FP64 oracle on the whole decode batch (every row), repeated
+    until about min_seconds of CPU work; returns (GB/s, seconds, threads,
+    passes)."""
+    s = case.spec
+    oc = _oracle_cache(case)
+    rows = [[b, h] for b in range(len(s.context_lens)) for h in range(s.num_q_heads)]
+    total, passes, used = 0.0, 0, 0
+    while passes < max_passes and (passes == 0 or total < min_seconds):
+        dt, used = _oracle_rows(oc, case, rows)
+        total += dt
+        passes += 1
+    nbytes = synth.kv_read_bytes(s) * passes
+    return nbytes / total / 1e9, total, used, passes
 
 
 def run_reference(args, rank: int):
+    """The reference arm: the FP64 oracle, as it stands, on the host cores.
+    Each step is a bounded sample of the decode batch, sized so that W + K
+    steps take about REFERENCE_BUDGET_S seconds: `rows_per_step` (sequence,
+    query head) rows taken round-robin over the whole batch."""
     if rank != 0:
         return
-    import oracle
     spec = synth.workload(DECODE_WORKLOAD)
     case = synth.make_case(spec)
-    nbytes, _, used, oc = oracle_decode_sample(case, 1)   # builds the oracle cache, warms up
+    oc = _oracle_cache(case)
+    all_rows = [[b, h] for b in range(len(spec.context_lens)) for h in range(spec.num_q_heads)]
+    t_row, used = _oracle_rows(oc, case, all_rows[:8])
+    t_row /= 8
+    n_calls = max(1, args.warmup + args.steps)
+    rows_per_step = int(max(1, min(len(all_rows), REFERENCE_BUDGET_S / n_calls / max(t_row, 1e-6))))
     times = []
-    for i in range(args.warmup + args.steps):
-        b = i % len(spec.context_lens)
-        rows = np.array([[b, h] for h in range(spec.num_q_heads)], np.int32)
-        t0 = time.perf_counter()
-        oracle.paged_attention(oc, _bits16(case.q), case.cu_seqlens_q.numpy(),
-                               case.context_lens.numpy(), case.block_table.numpy(),
-                               case.softmax_scale, rows=rows)
+    for i in range(n_calls):
+        k0 = (i * rows_per_step) % len(all_rows)
+        rows = [all_rows[(k0 + r) % len(all_rows)] for r in range(rows_per_step)]
+        dt, used = _oracle_rows(oc, case, rows)
         if i >= args.warmup:
-            times.append(time.perf_counter() - t0)
+            times.append(dt)
     t = sum(times) / len(times)
-    val = nbytes / t / 1e9
-    sample = ("each step: all 32 query heads of one of the 8 sequences "
-              "(1/8 of the batch, 33,554,432 KV bytes), FP64 oracle")
+    val = rows_per_step * _row_bytes(spec) / t / 1e9
+    sample = (f"each step: {rows_per_step} of the 256 (sequence, query head) rows of the "
+              f"batch-8 x 32K decode, round-robin; FP64 oracle; value = their share of the "
+              f"KV bytes / time")
     line = {
         "impl": "reference", "metric": METRIC, "value": val,
         "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -418,39 +443,76 @@ def main():
     dec_gbs = kv_bytes / (ms_dec * 1e-3) / 1e9
 
     # ---------------- end to end through the public API, host buffers ----------------
-    host = {k: inp[k].cpu().pin_memory() for k in ("q", "k_new", "v_new", "slot_new", "bt", "ctx")}
-    host_out = torch.empty(inp["out"].shape, dtype=inp["out"].dtype).pin_memory()
-    dev_in = {k: torch.empty_like(inp[k]) for k in host}
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = host_out.numel() * host_out.element_size()
+    # Every step uploads its inputs (new token's K/V and slots, Q, block table,
+    # context lengths) from pinned host memory and reads its output back.  The
+    # inputs sit back to back in one pinned buffer, so one copy moves them; two
+    # device copies of that buffer (and of the output) let step i+1's upload
+    # and step i's download run on their own streams while step i computes.
+    names = ("q", "k_new", "v_new", "slot_new", "bt", "ctx")
+    offs, total = {}, 0
+    for k in names:
+        nb = inp[k].numel() * inp[k].element_size()
+        offs[k] = (total, nb)
+        total += (nb + 255) // 256 * 256
+    host_in = torch.empty(total, dtype=torch.uint8).pin_memory()
+    for k, (o, nb) in offs.items():
+        host_in[o:o + nb].copy_(inp[k].reshape(-1).view(torch.uint8).cpu())
+    dev_in = [torch.empty(total, dtype=torch.uint8, device=device) for _ in range(2)]
+    views = [{k: buf[o:o + nb].view(inp[k].dtype).view(inp[k].shape)
+              for k, (o, nb) in offs.items()} for buf in dev_in]
+    dev_out = [torch.empty_like(inp["out"]) for _ in range(2)]
+    host_out = [torch.empty(inp["out"].shape, dtype=inp["out"].dtype).pin_memory()
+                for _ in range(2)]
+    h2d = sum(nb for _, nb in offs.values())
+    d2h = host_out[0].numel() * host_out[0].element_size()
+    up, down = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
+    copied = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    read = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step(cache):
-        with torch.cuda.stream(stream):
-            for k, t in host.items():
-                dev_in[k].copy_(t, non_blocking=True)
-            pk.kv_write_quant(cache, dev_in["k_new"], dev_in["v_new"], dev_in["slot_new"],
-                              stream=stream)
-            pk.paged_attn_decode(cache, dev_in["q"], dev_in["bt"], dev_in["ctx"], max_ctx, scale,
-                                 out=inp["out"], workspace=inp["ws"], stream=stream)
-            host_out.copy_(inp["out"], non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        if i >= 2:
+            up.wait_event(done[b])           # step i-2 finished with this input buffer
+        with torch.cuda.stream(up):
+            dev_in[b].copy_(host_in, non_blocking=True)
+        copied[b].record(up)
+        stream.wait_event(copied[b])
+        if i >= 2:
+            stream.wait_event(read[b])       # step i-2's output has been read back
+        d = views[b]
+        pk.kv_write_quant(caches[i % 2], d["k_new"], d["v_new"], d["slot_new"], stream=stream)
+        pk.paged_attn_decode(caches[i % 2], d["q"], d["bt"], d["ctx"], max_ctx, scale,
+                             out=dev_out[b], workspace=inp["ws"], stream=stream)
+        done[b].record(stream)
+        down.wait_event(done[b])
+        with torch.cuda.stream(down):
+            host_out[b].copy_(dev_out[b], non_blocking=True)
+        read[b].record(down)
 
-    for i in range(10):
-        e2e_step(caches[i % 2])
+    def e2e_steps(n):
+        up.wait_stream(stream)
+        down.wait_stream(stream)
+        for i in range(n):
+            e2e_step(i)
+        stream.wait_stream(up)
+        stream.wait_stream(down)
+
+    # The loop is captured once in a CUDA graph of E2E_GRAPH_STEPS steps (the
+    # uploads and downloads become memcpy nodes on the forked streams), as a
+    # serving loop would, so the host's per-call overhead is not what is timed.
+    with torch.cuda.stream(stream):
+        e2e_steps(4)
     torch.cuda.synchronize()
-    n_e2e = max(2, args.e2e_steps)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if barrier:
-        barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for i in range(n_e2e):
-        e2e_step(caches[i % 2])
-    e1.record(stream)
-    torch.cuda.synchronize()
-    if barrier:
-        barrier()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e)
+    g_e2e = capture(lambda: e2e_steps(E2E_GRAPH_STEPS), stream)
+    n_rep = max(1, args.e2e_steps // E2E_GRAPH_STEPS)
+    n_e2e = n_rep * E2E_GRAPH_STEPS
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g_e2e.replay()
+    ms_e2e = max_over_ranks(time_graph(g_e2e, n_rep, stream, barrier) / E2E_GRAPH_STEPS)
     e2e_val = world * kv_bytes / (ms_e2e * 1e-3) / 1e9
+    ok_out = bool(torch.equal(host_out[(n_e2e - 1) % 2].to(device), dev_out[(n_e2e - 1) % 2]))
 
     # ---------------- secondary: causal prefill 8K ----------------
     secondary = None
@@ -497,10 +559,10 @@ def main():
     # ---------------- CPU baseline (oracle, rank 0, N = 1) ----------------
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        nb, dt, used, _ = oracle_decode_sample(case, 2)
-        cpu = {"value": nb / dt / 1e9, "unit": "GB/s", "cores": used, "kind": "oracle",
-               "sample": "all 32 query heads of 2 of the 8 sequences (64 of 256 rows, "
-                         f"{nb} KV bytes), FP64 oracle, {dt:.1f} s"}
+        gbs, dt, used, passes = oracle_decode_sample(case)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle",
+               "sample": f"the whole batch-8 x 32K decode (all 256 rows, 268,435,456 KV "
+                         f"bytes) x {passes} passes, FP64 oracle, {dt:.1f} s"}
 
     launches_per_step = 2 + (1 if plan_splits else 0)
     traffic = decode_traffic_from_profile()
@@ -513,7 +575,11 @@ def main():
         "config": decode_config(spec, world),
         "clocks": clk.summary(),
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e,
+                "pipelining": "per step one pinned upload (own stream) and one download (third "
+                              "stream), double-buffered device inputs/outputs; 8 steps per "
+                              "CUDA graph replay",
+                "last_output_read_back_matches": ok_out},
         "gpu_launches": launches_per_step * steps,
         "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": dec_gbs / hbm_peak, "traffic": traffic,
@@ -526,7 +592,7 @@ def main():
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g_step, g_dec, g_wr
+    del g_step, g_dec, g_wr, g_e2e
     if dist:
         dist.barrier()
         dist.destroy_process_group()
