@@ -556,7 +556,9 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
     const int rr = (int)(gw % p.rows);
     const int h = (int)((gw / p.rows) % p.num_kv_heads);
     const int b = (int)(gw / ((long long)p.rows * p.num_kv_heads));
+    // every global load of this row is issued before any is used
     const int ctx = p.context_lens[b];
+    const float vfac = p.v_scale ? __ldg(p.v_scale + h) : 1.0f;
     const int nblk = (ctx + p.block_size - 1) / p.block_size;
     const int nvalid = min(p.num_splits, (nblk + p.blocks_per_split - 1) / p.blocks_per_split);
     const size_t base = ((size_t)b * p.num_kv_heads + h) * p.num_splits * p.rows + rr;
@@ -599,7 +601,6 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
         }
         M = cm;
     }
-    const float vfac = p.v_scale ? __ldg(p.v_scale + h) : 1.0f;
     const int tq = rr / p.group, gq = rr % p.group;
     const size_t orow = ((size_t)b * p.q_len + tq) * p.num_q_heads + h * p.group + gq;
     __half2 lo = __floats2half2_rn(L > 0.0f ? O.x / L * vfac : 0.0f, L > 0.0f ? O.y / L * vfac : 0.0f);
