@@ -68,6 +68,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--only", choices=["decode", "prefill"], default=None)
+    ap.add_argument("--workload", type=int, default=None,
+                    help="with --only: the named workload to run (decode 1, 2, 5; prefill 3, 4)")
     return ap.parse_args()
 
 
@@ -235,14 +237,14 @@ def run_reference(args, rank: int):
 
 # -------------------------------------------------------------- GPU arm --
 
-def build_decode(case, device):
+def build_decode(case, device, copies: int = 2):
     import paged_quantized_kv_quant_b200 as pk
     s = case.spec
     B, ql, Hq, D = len(s.context_lens), s.q_lens[0], s.num_q_heads, s.head_dim
     k_all, v_all = case.k.to(device), case.v.to(device)
     sm_all = case.slot_mapping.to(device)
     caches = []
-    for _ in range(2):     # two copies: consecutive steps never share L2 lines
+    for _ in range(copies):   # two copies: consecutive steps never share L2 lines
         c = pk.PagedKVCache.allocate(s.kv_dtype, case.num_blocks, s.block_size,
                                      s.num_kv_heads, D, device=device,
                                      k_scale=case.k_scale, v_scale=case.v_scale)
@@ -338,13 +340,17 @@ def run_only(args):
     device = torch.device("cuda", 0)
     stream = torch.cuda.Stream(device=device)
     if args.only == "decode":
-        spec = synth.workload(DECODE_WORKLOAD)
+        spec = synth.workload(args.workload or DECODE_WORKLOAD)
         case = synth.make_case(spec)
-        caches, inp, max_ctx, _ = build_decode(case, device)
+        # two cache copies alternate when they are small; one copy of a
+        # cache larger than L2 already defeats it
+        copies = 2 if synth.kv_read_bytes(spec) < (1 << 30) else 1
+        caches, inp, max_ctx, _ = build_decode(case, device, copies=copies)
+        torch.cuda.empty_cache()   # keep only what the calls use on the device
         calls = [lambda c=c: decode_step(pk, c, inp, max_ctx, case.softmax_scale, write=False)
                  for c in caches]
     else:
-        spec = synth.workload(PREFILL_WORKLOAD)
+        spec = synth.workload(args.workload or PREFILL_WORKLOAD)
         case = synth.make_case(spec)
         c = pk.PagedKVCache.allocate(spec.kv_dtype, case.num_blocks, spec.block_size,
                                      spec.num_kv_heads, device=device,

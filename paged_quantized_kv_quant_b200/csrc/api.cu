@@ -295,11 +295,12 @@ pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void *q, void 
     p.rows_per_cta = plan.rows_per_cta;
     p.row_groups = plan.row_groups;
     p.num_splits = plan.num_splits;
-    p.blocks_per_split = plan.blocks_per_split;
+    p.uniform_splits = plan.uniform_splits;
+    p.uniform_bpc = plan.uniform_bpc;
     p.scale_log2 = softmax_scale * kLog2e;
     float *ws = static_cast<float *>(workspace);
-    const size_t n_rows_ws =
-        (size_t)batch * cache->num_kv_heads * plan.num_splits * p.rows;
+    const size_t n_rows_ws = (size_t)cache->num_kv_heads * plan.row_groups * plan.num_splits *
+                             plan.rows_per_cta;
     p.ws_o = plan.workspace_bytes ? ws : nullptr;
     p.ws_ml = plan.workspace_bytes ? ws + n_rows_ws * kHeadDim : nullptr;
     p.status = status_ptr();

@@ -8,7 +8,12 @@
 //
 // Work decomposition.  A CTA owns one (sequence, KV head, row group, split):
 // the rows are the q_len x G query rows that share the KV head (GQA packing),
-// the split is a contiguous range of cache blocks.  Each of its 4 warps
+// the split is a contiguous range of cache blocks.  Every (KV head, row group)
+// gets the same number C of CTA slots; slot c is mapped on the device, from
+// the context lengths, to a sequence and a split of it, each sequence getting
+// splits in proportion to its length (at least one), so that sequences of
+// different lengths still give every CTA about the same work.  Each of its 4
+// warps
 // streams whole cache blocks (block_size x 128 codes of K and of V, one
 // contiguous tile each) through a private ring of TMA stages: lane 0 issues a
 // 2-D tensor copy per tile with 128-byte swizzle, so the fragment loads below
@@ -192,6 +197,89 @@ __device__ __forceinline__ void pv_block(const uint8_t *vt, const uint16_t *st, 
     }
 }
 
+constexpr int kMinBlocksPerWarp = 3;   // shortest split: 3 cache blocks per warp
+
+// Blocks per split for C slots over `batch` sequences holding `total`
+// blocks, the longest `longest`: with C > batch, ceil(total / (C - batch))
+// (never below kMinBlocksPerWarp per warp) keeps sum_b max(1, ceil(n_b /
+// bpc)) <= total / bpc + batch <= C; with C == batch every sequence gets one.
+__host__ __device__ inline int split_blocks(long long total, int C, int batch, int longest)
+{
+    if (C <= batch)
+        return max(1, longest);
+    const long long v = (total + (C - batch) - 1) / (C - batch);
+    return (int)max(v, (long long)(kWarps * kMinBlocksPerWarp));
+}
+
+// Which (sequence, split) a CTA slot streams, or where a sequence's splits
+// are: computed by one warp from the context lengths, warp-uniform result.
+// Every sequence b gets nsplit_b = max(1, ceil(nblk_b / bpc)) consecutive
+// slots, bpc = split_blocks(total blocks, C, B, longest), which keeps the sum
+// within C.  The host uses split_blocks for its uniform-length guess.
+struct SplitInfo {
+    int b;        // sequence (-1: slot beyond the last split)
+    int split;    // split of that sequence
+    int nsplit;   // splits of that sequence
+    int first;    // slot of its first split
+    int ctx;      // its context length
+    int bpc;      // blocks per split
+};
+
+template <int BS>
+__device__ __forceinline__ int seq_blocks(const DecodeParams &p, int i)
+{
+    return i < p.batch ? (max(p.context_lens[i], 0) + BS - 1) / BS : 0;
+}
+
+// slot < 0: find sequence `seq`; otherwise find the sequence owning `slot`
+template <int BS>
+__device__ SplitInfo find_split(const DecodeParams &p, int slot, int seq)
+{
+    const int lane = threadIdx.x & 31;
+    const int C = p.num_splits;
+    long long total = 0;
+    int longest = 0;
+    int n0 = seq_blocks<BS>(p, lane);   // kept: most batches have at most 32 sequences
+    for (int base = 0; base < p.batch; base += 32) {
+        const int n = base == 0 ? n0 : seq_blocks<BS>(p, base + lane);
+        total += n;
+        longest = max(longest, n);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        total += __shfl_xor_sync(0xffffffffu, total, o);
+        longest = max(longest, __shfl_xor_sync(0xffffffffu, longest, o));
+    }
+    SplitInfo r{-1, 0, 0, 0, 0, split_blocks(total, C, p.batch, longest)};
+    int run = 0;   // slots taken by the sequences before this chunk
+    for (int base = 0; base < p.batch; base += 32) {
+        const int i = base + lane;
+        const int n = base == 0 ? n0 : seq_blocks<BS>(p, i);
+        const int ns = i < p.batch ? max(1, (n + r.bpc - 1) / r.bpc) : 0;
+        int incl = ns;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += v;
+        }
+        const int first = run + incl - ns;
+        const bool hit = i < p.batch && (slot >= 0 ? (slot >= first && slot < first + ns) : i == seq);
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (m) {
+            const int src = __ffs(m) - 1;
+            r.b = base + src;
+            r.first = __shfl_sync(0xffffffffu, first, src);
+            r.nsplit = __shfl_sync(0xffffffffu, ns, src);
+            r.split = slot >= 0 ? slot - r.first : 0;
+            r.ctx = max(p.context_lens[r.b], 0);
+            break;
+        }
+        run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    return r;
+}
+
 template <int KVT, int NT, int BS>
 __global__ void __launch_bounds__(kThreads)
 decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -210,10 +298,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     uint16_t *scales = reinterpret_cast<uint16_t *>(tiles + kWarps * S * C::kStageBytes);
     uint64_t *bars = reinterpret_cast<uint64_t *>(scales + kWarps * S * C::kScaleHalves);
 
-    const int split = blockIdx.x;
+    const int slot = blockIdx.x;
     const int h = blockIdx.y % p.num_kv_heads;
     const int rg = blockIdx.y / p.num_kv_heads;
-    const int b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
 
@@ -239,55 +326,79 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 
     if (device_wait_failed(p.status))
         return;
-    const int blk_begin = split * p.blocks_per_split;
-    // Block ids of this warp's first 64 iterations are loaded speculatively
-    // (every index stays inside the table row), in parallel with the context
-    // length, so the first copies wait for one memory round trip, not two.
-    const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq;
-    auto lblk = [&](int it) { return blk_begin + warp + kWarps * it; };
-    int win0 = lblk(lane) < p.max_blocks_per_seq ? __ldg(bt + lblk(lane)) : 0;
-    int win1 = lblk(32 + lane) < p.max_blocks_per_seq ? __ldg(bt + lblk(32 + lane)) : 0;
-    int win_base = 0;
-    const int ctx = p.context_lens[b];
-    const int nblk_seq = (ctx + BS - 1) / BS;
-    if (p.num_splits > 1 && blk_begin >= nblk_seq)
-        return;   // the merge kernel only reads splits that hold keys
-    const int nblk = max(0, min(nblk_seq, blk_begin + p.blocks_per_split) - blk_begin);
-    const int n_it = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
-
-    // ---- query fragments (B operand of S^T = K Q^T), loop invariant ----
+    // The block ids of this warp's first 64 iterations and the query rows are
+    // loaded for a guess of this slot's (sequence, split): the assignment all
+    // sequences at max_context_len would give.  They are loaded while the
+    // real assignment is computed from the context lengths, and reloaded
+    // only when the guess was wrong (different lengths), so that with equal
+    // lengths the first copies wait for one memory round trip, not two.
+    int b = min(slot / p.uniform_splits, p.batch - 1);
+    int blk_begin = (slot - b * p.uniform_splits) * p.uniform_bpc;
     const int h0 = h * p.group;
+    int win0, win1;
+    int win_base = 0;
+    auto lblk = [&](int it) { return blk_begin + warp + kWarps * it; };
+    auto load_window = [&]() {   // every index stays inside the table row
+        const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq;
+        win0 = lblk(lane) < p.max_blocks_per_seq ? __ldg(bt + lblk(lane)) : 0;
+        win1 = lblk(32 + lane) < p.max_blocks_per_seq ? __ldg(bt + lblk(32 + lane)) : 0;
+    };
+    // query fragments (B operand of S^T = K Q^T), loop invariant
     uint32_t qf[NT][8][2];
+    auto load_q = [&]() {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int r = rg * RC + nt * 8 + g;
+            uint32_t u[16];
+            if (r < p.rows) {
+                const int tq = r / p.group, gq = r % p.group;
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    p.q + (((size_t)b * p.q_len + tq) * p.num_q_heads + h0 + gq) * kHeadDim +
+                    32 * t);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    uint4 w = __ldg(src + i);
+                    u[4 * i] = w.x, u[4 * i + 1] = w.y, u[4 * i + 2] = w.z, u[4 * i + 3] = w.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    u[i] = 0u;
+            }
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                qf[nt][ks][0] = u[2 * ks];       // d = 32t + 4ks + {0,1}
+                qf[nt][ks][1] = u[2 * ks + 1];   // d = 32t + 4ks + {2,3}
+            }
+        }
+    };
+    load_window();
+    load_q();
+    const SplitInfo si = find_split<BS>(p, slot, -1);
+    if (si.b < 0)
+        return;   // a slot past the last split: no work
+    const int real_begin = si.split * si.bpc;
+    if (si.b != b || real_begin != blk_begin) {
+        const bool new_seq = si.b != b;
+        b = si.b;
+        blk_begin = real_begin;
+        load_window();
+        if (new_seq)
+            load_q();
+    }
+    const int ctx = si.ctx;
+    const int nblk_seq = (ctx + BS - 1) / BS;
+    const int nblk = max(0, min(nblk_seq, blk_begin + si.bpc) - blk_begin);
+    const int n_it = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
+    const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq;
     int pos[NT][2];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        const int r = rg * RC + nt * 8 + g;
-        uint32_t u[16];
-        if (r < p.rows) {
-            const int tq = r / p.group, gq = r % p.group;
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                p.q + (((size_t)b * p.q_len + tq) * p.num_q_heads + h0 + gq) * kHeadDim + 32 * t);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint4 w = __ldg(src + i);
-                u[4 * i] = w.x, u[4 * i + 1] = w.y, u[4 * i + 2] = w.z, u[4 * i + 3] = w.w;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                u[i] = 0u;
-        }
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            qf[nt][ks][0] = u[2 * ks];       // d = 32t + 4ks + {0,1}
-            qf[nt][ks][1] = u[2 * ks + 1];   // d = 32t + 4ks + {2,3}
-        }
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             const int rr = rg * RC + nt * 8 + 2 * t + i;
             pos[nt][i] = rr < p.rows ? ctx - p.q_len + rr / p.group : ctx - 1;
         }
-    }
 
     float kfac = p.scale_log2;
     if constexpr (KVT == kKvFp8)
@@ -519,15 +630,14 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
             L += sl[w * RC + r] * e;
             O += so[(w * RC + r) * kHeadDim + d] * e;
         }
-        if (p.num_splits == 1) {
+        if (si.nsplit == 1) {
             const int tq = rr / p.group, gq = rr % p.group;
             const size_t orow = ((size_t)b * p.q_len + tq) * p.num_q_heads + h0 + gq;
             p.out[orow * kHeadDim + d] = __float2half_rn(L > 0.0f ? O / L * vfac : 0.0f);
             if (d == 0 && p.lse)
                 p.lse[orow] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
         } else {
-            const size_t wrow =
-                (((size_t)b * p.num_kv_heads + h) * p.num_splits + split) * p.rows + rr;
+            const size_t wrow = ((size_t)blockIdx.y * p.num_splits + slot) * RC + r;
             p.ws_o[wrow * kHeadDim + d] = O;
             if (d == 0)
                 *reinterpret_cast<float2 *>(p.ws_ml + wrow * 2) = make_float2(M, L);
@@ -540,11 +650,11 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 // The splits are taken kMergeChunk at a time: every lane issues the loads of
 // a whole chunk (the (m, l) pairs, the same for all lanes, and its float4 of
 // each O row) before using any, so a chunk costs one memory round trip; the
-// chunks are combined online.  The first chunk is loaded without waiting for
-// the context length (splits past the last one that holds keys are loaded
-// from the workspace but not used).
+// chunks are combined online.  A sequence that a single split covered was
+// finished by that split.
 constexpr int kMergeChunk = 16;
 
+template <int BS>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -556,35 +666,41 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
     const int rr = (int)(gw % p.rows);
     const int h = (int)((gw / p.rows) % p.num_kv_heads);
     const int b = (int)(gw / ((long long)p.rows * p.num_kv_heads));
-    // every global load of this row is issued before any is used
-    const int ctx = p.context_lens[b];
     const float vfac = p.v_scale ? __ldg(p.v_scale + h) : 1.0f;
-    const int nblk = (ctx + p.block_size - 1) / p.block_size;
-    const int nvalid = min(p.num_splits, (nblk + p.blocks_per_split - 1) / p.blocks_per_split);
-    const size_t base = ((size_t)b * p.num_kv_heads + h) * p.num_splits * p.rows + rr;
-    float M = -INFINITY, L = 0.0f;
-    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < p.num_splits; s0 += kMergeChunk) {
-        if (s0 > 0 && s0 >= nvalid)
-            break;
-        float2 ml[kMergeChunk];
-        float4 v[kMergeChunk];
+    // slots first .. first + nsplit - 1 of unit (row group, KV head) y
+    const int y = (rr / p.rows_per_cta) * p.num_kv_heads + h;
+    const size_t row0 = (size_t)y * p.num_splits * p.rows_per_cta + rr % p.rows_per_cta;
+    const size_t stride = p.rows_per_cta;
+    float2 ml[kMergeChunk];
+    float4 v[kMergeChunk];
+    auto load_chunk = [&](int first, int nsplit, int s0) {
 #pragma unroll
         for (int k = 0; k < kMergeChunk; ++k) {
             ml[k] = make_float2(-INFINITY, 0.0f);
             v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (s0 + k < p.num_splits) {
-                const size_t wrow = base + (size_t)(s0 + k) * p.rows;
+            if (s0 + k < nsplit && first + s0 + k < p.num_splits) {
+                const size_t wrow = row0 + (size_t)(first + s0 + k) * stride;
                 ml[k] = *reinterpret_cast<const float2 *>(p.ws_ml + wrow * 2);
                 v[k] = reinterpret_cast<const float4 *>(p.ws_o + wrow * kHeadDim)[lane];
             }
         }
-#pragma unroll
-        for (int k = 0; k < kMergeChunk; ++k)
-            if (s0 + k >= nvalid) {
-                ml[k] = make_float2(-INFINITY, 0.0f);
-                v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+    };
+    // The first chunk is loaded for the slots all sequences at
+    // max_context_len would give, while the real slots are computed from the
+    // context lengths; it is reloaded only when they differ.
+    const int gfirst = b * p.uniform_splits;
+    load_chunk(gfirst, p.uniform_splits, 0);
+    const SplitInfo si = find_split<BS>(p, -1, b);
+    if (si.nsplit <= 1)
+        return;   // a single split wrote the final row itself
+    if (si.first != gfirst || si.nsplit != p.uniform_splits)
+        load_chunk(si.first, si.nsplit, 0);
+    const int nvalid = si.nsplit;
+    float M = -INFINITY, L = 0.0f;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < nvalid; s0 += kMergeChunk) {
+        if (s0 > 0)
+            load_chunk(si.first, nvalid, s0);
         float cm = M;
 #pragma unroll
         for (int k = 0; k < kMergeChunk; ++k)
@@ -623,7 +739,7 @@ cudaError_t launch_split(const DecodeParams &p, const CUtensorMap &kmap, const C
     if (e != cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.num_splits, p.num_kv_heads * p.row_groups, p.batch);
+    cfg.gridDim = dim3(p.num_splits, p.num_kv_heads * p.row_groups, 1);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -706,17 +822,16 @@ bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv
     plan->rows_per_cta = 8 * plan->nt;
     plan->row_groups = (rows + plan->rows_per_cta - 1) / plan->rows_per_cta;
     const int max_blocks = (max_context_len + block_size - 1) / block_size;
-    const long long units = (long long)batch * num_kv_heads * plan->row_groups;
-    // At most `ctas_per_sm` CTAs on every SM (3, or what fits), all resident
-    // in one wave, with the same number of blocks each: rounding the split
-    // count up instead would put one more CTA on some SMs, and those SMs'
-    // CTAs would all finish last (a memory-bound CTA gets a share of its
-    // SM's bandwidth).  More resident CTAs keep more copies in flight.  Never
-    // split below kMinBlocksPerWarp blocks per warp: short splits pay the
-    // fixed start-up and merge costs for little streaming.
+    const int units = num_kv_heads * plan->row_groups;   // grid y: (row group, KV head)
+    // C CTA slots per unit, at most `ctas_per_sm` CTAs on every SM (3, or
+    // what fits), all resident in one wave, each slot given about the same
+    // number of blocks on the device.  Rounding the count up instead would
+    // put one more CTA on some SMs, and those SMs' CTAs would all finish last
+    // (a memory-bound CTA gets a share of its SM's bandwidth); more resident
+    // CTAs keep more copies in flight.  At least one slot per sequence, and
+    // no more slots than splits of kMinBlocksPerWarp blocks per warp.
     // PKVQ_DECODE_CTAS_PER_SM (1..16) replaces the target as given, even
     // beyond what fits in one wave.
-    constexpr int kMinBlocksPerWarp = 3;
     int ctas_per_sm = min(3, split_occupancy(kv_dtype, plan->nt, block_size));
     if (const char *env = getenv("PKVQ_DECODE_CTAS_PER_SM")) {
         const int v = atoi(env);
@@ -724,17 +839,19 @@ bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv
             ctas_per_sm = v;
     }
     const long long target = (long long)ctas_per_sm * device_sm_count();
-    long long splits = target / units;
-    const long long max_splits =
-        max(1, max_blocks / (kWarps * kMinBlocksPerWarp));
-    splits = max(1LL, min(splits, max_splits));
-    int bps = max_blocks > 0 ? (int)((max_blocks + splits - 1) / splits) : 1;
-    splits = max_blocks > 0 ? (max_blocks + bps - 1) / bps : 1;
-    plan->num_splits = (int)splits;
-    plan->blocks_per_split = bps;
-    plan->workspace_bytes =
-        splits > 1 ? (size_t)batch * num_kv_heads * splits * rows * (kHeadDim + 2) * sizeof(float)
-                   : 0;
+    long long C = max((long long)batch, target / units);
+    const long long useful =
+        (long long)batch * max(1, max_blocks / (kWarps * kMinBlocksPerWarp));
+    C = min(C, max((long long)batch, useful));
+    if (C > (1LL << 30))
+        return false;
+    plan->num_splits = (int)C;
+    // the split every slot gets when all sequences hold max_context_len tokens
+    plan->uniform_bpc = split_blocks((long long)batch * max_blocks, (int)C, batch, max_blocks);
+    plan->uniform_splits = max(1, (max_blocks + plan->uniform_bpc - 1) / plan->uniform_bpc);
+    plan->workspace_bytes = C > batch ? (size_t)units * C * plan->rows_per_cta *
+                                            (kHeadDim + 2) * sizeof(float)
+                                      : 0;
     return true;
 }
 
@@ -748,8 +865,8 @@ cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_
     else
         e = plan.nt == 1 ? launch_bs<kKvInt8, 1>(p, kmap, vmap, stream)
                          : launch_bs<kKvInt8, 2>(p, kmap, vmap, stream);
-    if (e != cudaSuccess || p.num_splits == 1)
-        return e;
+    if (e != cudaSuccess || p.num_splits <= p.batch)
+        return e;   // one slot per sequence: every split wrote its final rows
     const long long rows_total = (long long)p.batch * p.num_kv_heads * p.rows;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((rows_total + 3) / 4));
@@ -761,7 +878,12 @@ cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_merge_kernel, p);
+    switch (p.block_size) {
+    case 16: return cudaLaunchKernelEx(&cfg, decode_merge_kernel<16>, p);
+    case 32: return cudaLaunchKernelEx(&cfg, decode_merge_kernel<32>, p);
+    case 64: return cudaLaunchKernelEx(&cfg, decode_merge_kernel<64>, p);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace pkvq

@@ -39,17 +39,21 @@ struct DecodeParams {
     int rows;            // q_len * group rows per (sequence, KV head)
     int rows_per_cta;    // 8 * NT
     int row_groups;      // ceil(rows / rows_per_cta)
-    int num_splits;      // splits of the block range per (sequence, KV head)
-    int blocks_per_split;
+    int num_splits;      // C: CTA slots per (row group, KV head), mapped to
+                         // (sequence, split) on the device from the lengths
+    int uniform_splits;  // splits per sequence when all hold max_context_len
+    int uniform_bpc;     // blocks per split in that case
     float scale_log2;    // softmax_scale * log2(e)
-    float *ws_o;         // [B][Hkv][splits][rows][128] fp32, unnormalised
-    float *ws_ml;        // [B][Hkv][splits][rows][2] fp32 (max in log2 units, sum)
+    float *ws_o;         // [row groups x Hkv][C][rows_per_cta][128] fp32, unnormalised
+    float *ws_ml;        // [row groups x Hkv][C][rows_per_cta][2] fp32 (log2 max, sum)
     uint32_t *status;
 };
 
 struct DecodePlan {
     int nt;              // n8 row tiles per CTA (1 or 2)
-    int rows_per_cta, row_groups, num_splits, blocks_per_split;
+    int rows_per_cta, row_groups;
+    int num_splits;                     // C slots per (row group, KV head)
+    int uniform_splits, uniform_bpc;    // the assignment with equal lengths
     size_t workspace_bytes;
 };
 
