@@ -28,6 +28,11 @@ CASES = [
     (FP8, 8, 1, [4099], 4, 16),             # q_len 4, G 8 -> 32 rows
     (FP8, 32, 4, [16384], 1, 16),           # long: many splits
     (INT8, 8, 2, [20000, 3], 2, 16),
+    # splits in proportion to length: one long sequence among very short ones
+    (FP8, 8, 2, [65536, 1, 16, 17, 4096, 300], 1, 16),
+    (INT8, 16, 2, [3000, 40000, 5], 2, 16),
+    # more than 32 sequences: the slot map is scanned in several warp chunks
+    (FP8, 8, 2, [(i * 977) % 3001 + 1 for i in range(40)], 1, 16),
 ]
 
 
