@@ -297,6 +297,8 @@ pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void *q, void 
     p.num_splits = plan.num_splits;
     p.uniform_splits = plan.uniform_splits;
     p.uniform_bpc = plan.uniform_bpc;
+    p.split_min_blocks = plan.split_min_blocks;
+    p.split_gran = plan.split_gran;
     p.scale_log2 = softmax_scale * kLog2e;
     float *ws = static_cast<float *>(workspace);
     const size_t n_rows_ws = (size_t)cache->num_kv_heads * plan.row_groups * plan.num_splits *

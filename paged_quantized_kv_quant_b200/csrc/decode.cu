@@ -35,6 +35,7 @@
 // small probabilities never meet small scales in fp16).
 #include "common.cuh"
 #include "internal.h"
+#include "split_map.cuh"
 
 #include <math.h>
 
@@ -198,87 +199,6 @@ __device__ __forceinline__ void pv_block(const uint8_t *vt, const uint16_t *st, 
 }
 
 constexpr int kMinBlocksPerWarp = 3;   // shortest split: 3 cache blocks per warp
-
-// Blocks per split for C slots over `batch` sequences holding `total`
-// blocks, the longest `longest`: with C > batch, ceil(total / (C - batch))
-// (never below kMinBlocksPerWarp per warp) keeps sum_b max(1, ceil(n_b /
-// bpc)) <= total / bpc + batch <= C; with C == batch every sequence gets one.
-__host__ __device__ inline int split_blocks(long long total, int C, int batch, int longest)
-{
-    if (C <= batch)
-        return max(1, longest);
-    const long long v = (total + (C - batch) - 1) / (C - batch);
-    return (int)max(v, (long long)(kWarps * kMinBlocksPerWarp));
-}
-
-// Which (sequence, split) a CTA slot streams, or where a sequence's splits
-// are: computed by one warp from the context lengths, warp-uniform result.
-// Every sequence b gets nsplit_b = max(1, ceil(nblk_b / bpc)) consecutive
-// slots, bpc = split_blocks(total blocks, C, B, longest), which keeps the sum
-// within C.  The host uses split_blocks for its uniform-length guess.
-struct SplitInfo {
-    int b;        // sequence (-1: slot beyond the last split)
-    int split;    // split of that sequence
-    int nsplit;   // splits of that sequence
-    int first;    // slot of its first split
-    int ctx;      // its context length
-    int bpc;      // blocks per split
-};
-
-template <int BS>
-__device__ __forceinline__ int seq_blocks(const DecodeParams &p, int i)
-{
-    return i < p.batch ? (max(p.context_lens[i], 0) + BS - 1) / BS : 0;
-}
-
-// slot < 0: find sequence `seq`; otherwise find the sequence owning `slot`
-template <int BS>
-__device__ SplitInfo find_split(const DecodeParams &p, int slot, int seq)
-{
-    const int lane = threadIdx.x & 31;
-    const int C = p.num_splits;
-    long long total = 0;
-    int longest = 0;
-    int n0 = seq_blocks<BS>(p, lane);   // kept: most batches have at most 32 sequences
-    for (int base = 0; base < p.batch; base += 32) {
-        const int n = base == 0 ? n0 : seq_blocks<BS>(p, base + lane);
-        total += n;
-        longest = max(longest, n);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        total += __shfl_xor_sync(0xffffffffu, total, o);
-        longest = max(longest, __shfl_xor_sync(0xffffffffu, longest, o));
-    }
-    SplitInfo r{-1, 0, 0, 0, 0, split_blocks(total, C, p.batch, longest)};
-    int run = 0;   // slots taken by the sequences before this chunk
-    for (int base = 0; base < p.batch; base += 32) {
-        const int i = base + lane;
-        const int n = base == 0 ? n0 : seq_blocks<BS>(p, i);
-        const int ns = i < p.batch ? max(1, (n + r.bpc - 1) / r.bpc) : 0;
-        int incl = ns;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o)
-                incl += v;
-        }
-        const int first = run + incl - ns;
-        const bool hit = i < p.batch && (slot >= 0 ? (slot >= first && slot < first + ns) : i == seq);
-        const unsigned m = __ballot_sync(0xffffffffu, hit);
-        if (m) {
-            const int src = __ffs(m) - 1;
-            r.b = base + src;
-            r.first = __shfl_sync(0xffffffffu, first, src);
-            r.nsplit = __shfl_sync(0xffffffffu, ns, src);
-            r.split = slot >= 0 ? slot - r.first : 0;
-            r.ctx = max(p.context_lens[r.b], 0);
-            break;
-        }
-        run += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    return r;
-}
 
 template <int KVT, int NT, int BS>
 __global__ void __launch_bounds__(kThreads)
@@ -818,11 +738,20 @@ bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv
         return false;
     const int group = num_q_heads / num_kv_heads;
     const int rows = q_len * group;
-    plan->nt = rows <= 8 ? 1 : 2;
-    plan->rows_per_cta = 8 * plan->nt;
+    // More than 16 rows per KV head (up to 128): the tensor-core kernel, one
+    // CTA for all rows, so every code is fetched and converted once; the
+    // mma.sync kernel would split the rows into groups that each convert it.
+    plan->tc = rows > 16 && rows <= 128;
+    plan->nt = plan->tc ? 0 : (rows <= 8 ? 1 : 2);
+    plan->rows_per_cta = plan->tc ? rows : 8 * plan->nt;
     plan->row_groups = (rows + plan->rows_per_cta - 1) / plan->rows_per_cta;
     const int max_blocks = (max_context_len + block_size - 1) / block_size;
     const int units = num_kv_heads * plan->row_groups;   // grid y: (row group, KV head)
+    // splits: tensor-core kernel in whole 64-key tiles, at least 4 of them;
+    // mma.sync kernel at least kMinBlocksPerWarp blocks per warp
+    const int min_blocks = plan->tc ? 4 * (64 / block_size) : kWarps * kMinBlocksPerWarp;
+    plan->split_min_blocks = min_blocks;
+    plan->split_gran = plan->tc ? 64 / block_size : 1;
     // C CTA slots per unit, at most `ctas_per_sm` CTAs on every SM (3, or
     // what fits), all resident in one wave, each slot given about the same
     // number of blocks on the device.  Rounding the count up instead would
@@ -832,7 +761,8 @@ bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv
     // no more slots than splits of kMinBlocksPerWarp blocks per warp.
     // PKVQ_DECODE_CTAS_PER_SM (1..16) replaces the target as given, even
     // beyond what fits in one wave.
-    int ctas_per_sm = min(3, split_occupancy(kv_dtype, plan->nt, block_size));
+    // (the tensor-core kernel takes most of an SM's shared memory: one CTA)
+    int ctas_per_sm = plan->tc ? 1 : min(3, split_occupancy(kv_dtype, plan->nt, block_size));
     if (const char *env = getenv("PKVQ_DECODE_CTAS_PER_SM")) {
         const int v = atoi(env);
         if (v >= 1 && v <= 16)
@@ -840,14 +770,14 @@ bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv
     }
     const long long target = (long long)ctas_per_sm * device_sm_count();
     long long C = max((long long)batch, target / units);
-    const long long useful =
-        (long long)batch * max(1, max_blocks / (kWarps * kMinBlocksPerWarp));
+    const long long useful = (long long)batch * max(1, max_blocks / min_blocks);
     C = min(C, max((long long)batch, useful));
     if (C > (1LL << 30))
         return false;
     plan->num_splits = (int)C;
     // the split every slot gets when all sequences hold max_context_len tokens
-    plan->uniform_bpc = split_blocks((long long)batch * max_blocks, (int)C, batch, max_blocks);
+    plan->uniform_bpc = split_blocks((long long)batch * max_blocks, (int)C, batch, max_blocks,
+                                     plan->split_min_blocks, plan->split_gran);
     plan->uniform_splits = max(1, (max_blocks + plan->uniform_bpc - 1) / plan->uniform_bpc);
     plan->workspace_bytes = C > batch ? (size_t)units * C * plan->rows_per_cta *
                                             (kHeadDim + 2) * sizeof(float)
@@ -859,7 +789,9 @@ cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_
                           const CUtensorMap &kmap, const CUtensorMap &vmap, cudaStream_t stream)
 {
     cudaError_t e;
-    if (kv_dtype == kKvFp8)
+    if (plan.tc)
+        e = launch_decode_tc(p, kv_dtype, kmap, vmap, stream);
+    else if (kv_dtype == kKvFp8)
         e = plan.nt == 1 ? launch_bs<kKvFp8, 1>(p, kmap, vmap, stream)
                          : launch_bs<kKvFp8, 2>(p, kmap, vmap, stream);
     else

@@ -43,6 +43,7 @@ struct DecodeParams {
                          // (sequence, split) on the device from the lengths
     int uniform_splits;  // splits per sequence when all hold max_context_len
     int uniform_bpc;     // blocks per split in that case
+    int split_min_blocks, split_gran;   // shortest split; split sizes are multiples of gran
     float scale_log2;    // softmax_scale * log2(e)
     float *ws_o;         // [row groups x Hkv][C][rows_per_cta][128] fp32, unnormalised
     float *ws_ml;        // [row groups x Hkv][C][rows_per_cta][2] fp32 (log2 max, sum)
@@ -54,6 +55,8 @@ struct DecodePlan {
     int rows_per_cta, row_groups;
     int num_splits;                     // C slots per (row group, KV head)
     int uniform_splits, uniform_bpc;    // the assignment with equal lengths
+    int split_min_blocks, split_gran;
+    bool tc;                            // tensor-core kernel: all rows of a KV head in one CTA
     size_t workspace_bytes;
 };
 
@@ -61,6 +64,10 @@ struct DecodePlan {
 // kKvInt8, whose kernels differ in registers and so in occupancy).
 bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv_heads,
                  int block_size, int max_context_len, DecodePlan *plan);
+
+// The tensor-core decode kernel (all rows of a KV head in one CTA).
+cudaError_t launch_decode_tc(const DecodeParams &p, int kv_dtype, const CUtensorMap &kmap,
+                             const CUtensorMap &vmap, cudaStream_t stream);
 
 cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_dtype,
                           const CUtensorMap &kmap, const CUtensorMap &vmap,
