@@ -130,11 +130,15 @@ PKVQ_API size_t pkvq_decode_workspace_bytes(int32_t batch, int32_t q_len, int32_
  *                 <= max_context_len and <= max_blocks_per_seq * block_size.
  *   max_context_len  host-side upper bound of context_lens; sizes the split
  *                 plan (must match the value given to the workspace query).
+ *                 The kernels split each sequence's tokens over CTAs in
+ *                 proportion to its own context length, read on the device.
  *   softmax_scale scores are softmax_scale * q . k_dequantized.
  *   workspace     device scratch of at least pkvq_decode_workspace_bytes();
  *                 contents need not be initialised.  Calls that overlap on
  *                 the device must not share a workspace.
  * num_q_heads must be a multiple of num_kv_heads with a group of at most 16.
+ * Up to 16 query rows per KV head (q_len x group) run on mma.sync tiles;
+ * 17 to 128 rows run all rows of a KV head in one tcgen05 CTA.
  */
 PKVQ_API pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void *q, void *out,
                                    float *lse_out, const int32_t *block_table,
