@@ -315,6 +315,22 @@ def decode_sources_digest() -> str:
     return h.hexdigest()[:16]
 
 
+def reduce_max(x: float, dist=None, device=None) -> float:
+    """Max of x over all ranks of the process group (x itself without one):
+    every multi-GPU time is the slowest rank's."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, bytes_per_rank: float, ms_max: float) -> float:
+    """Whole-job GB/s under weak scaling: every rank reads its own batch's
+    bytes in the slowest rank's time."""
+    return world * bytes_per_rank / (ms_max * 1e-3) / 1e9
+
+
 def decode_traffic_from_profile():
     """DRAM bytes (read + write) of one decode call, split and merge kernels,
     from the committed ncu summary; None when the summary is missing or was
@@ -405,11 +421,7 @@ def main():
     barrier = (lambda: dist.barrier()) if dist else None
 
     def max_over_ranks(x: float) -> float:
-        if not dist:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, dist, device)
 
     # ---------------- decode workload ----------------
     spec = synth.workload(DECODE_WORKLOAD)
@@ -445,7 +457,7 @@ def main():
             g_dec.replay()
     ms_dec = max_over_ranks(time_graph(g_dec, reps, stream, barrier) / 2)
     ms_wr = max_over_ranks(time_graph(g_wr, reps, stream, barrier) / 2)
-    value = world * kv_bytes / (ms_step * 1e-3) / 1e9
+    value = job_throughput(world, kv_bytes, ms_step)
     dec_gbs = kv_bytes / (ms_dec * 1e-3) / 1e9
 
     # ---------------- end to end through the public API, host buffers ----------------
@@ -517,7 +529,7 @@ def main():
         for _ in range(3):
             g_e2e.replay()
     ms_e2e = max_over_ranks(time_graph(g_e2e, n_rep, stream, barrier) / E2E_GRAPH_STEPS)
-    e2e_val = world * kv_bytes / (ms_e2e * 1e-3) / 1e9
+    e2e_val = job_throughput(world, kv_bytes, ms_e2e)
     ok_out = bool(torch.equal(host_out[(n_e2e - 1) % 2].to(device), dev_out[(n_e2e - 1) % 2]))
 
     # ---------------- secondary: causal prefill 8K ----------------
