@@ -20,16 +20,17 @@
 //
 // Warp roles (12 warps; the softmax warps form one aligned group of four, as
 // each warp reaches only the tensor-memory lanes 32 * (warp % 4) + 0..31):
-//   warps 0-3  dequant: code tiles -> fp16 K/V tiles in the 128-byte-swizzled
-//              layout [d half][key][64 d] (the K-major B operand of Q K^T and
-//              the MN-major B operand of P V).  Warps 0-1 convert K, warps
-//              2-3 V, one key row per thread: with one query tile, nothing
-//              else shares the conversion of a tile, so it takes four warps
-//              to keep pace with the softmax.
+//   warps 0-3, 6-7  dequant: code tiles -> fp16 K/V tiles in the
+//              128-byte-swizzled layout [d half][key][64 d] (the K-major B
+//              operand of Q K^T and the MN-major B operand of P V), one key
+//              row per thread: warps 0-1 convert d 0-63 of K, warps 6-7 d
+//              64-127 of K, warps 2-3 all of V.  With one query tile nothing
+//              else shares the conversion of a tile, so it takes six warps to
+//              keep pace with the softmax; K is split further because Q K^T
+//              of a tile waits for it.
 //   warp 4     TMA producer: one 2-D box per cache block into a 5-stage ring.
 //   warp 5     TMEM allocation; the whole warp runs the issue loop, one
 //              elected lane issues each tcgen05 instruction.
-//   warps 6-7  idle.
 //   warps 8-11 softmax, thread i owns row i: Q row into tensor memory, S row
 //              read with tcgen05.ld, causal mask where a tile can cross a
 //              row's position, FP32 running max/sum, fp16 P row written over
@@ -58,7 +59,9 @@ constexpr float kLn2 = 0.693147180559945309f;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
 constexpr int kWarpTma = 4;
 constexpr int kWarpMma = 5;
-constexpr int kDequantWarps = 4;
+constexpr int kDequantWarps = 6;   // warps 0-3 and 6-7
+
+__device__ __forceinline__ bool is_dequant_warp(int w) { return w < 4 || w == 6 || w == 7; }
 constexpr int kSoftmaxWarp0 = 8;
 
 // tensor memory: S/P buffers 0 and 1 (P in the first 32 columns of its
@@ -324,10 +327,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             mma_commit_elect(bars.mma_done);
             warp_wait(bars.mma_done, 0, p.status);
         }
-    } else if (warp < kDequantWarps) {
+    } else if (is_dequant_warp(warp)) {
         // ------------------------------------------------------ dequant --
         const int row = (warp & 1) * 32 + lane;   // key row of this thread
-        const int isv = warp >> 1;                // 0: K, 1: V
+        const int isv = (warp == 2 || warp == 3) ? 1 : 0;   // 0: K (warps 0, 1, 6, 7), 1: V
+        const int c0 = warp >= 6 ? 4 : 0;         // first 16-byte chunk of the row
+        const int nch = isv ? 8 : 4;              // chunks this warp converts
         const float kfac = p.scale_log2;
         for (int j = 0; j < ntiles; ++j) {
             const int s = j % kCodeStages, bj = j % kKVBufs;
@@ -346,9 +351,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 const uint32_t sc = scl[64 + row];   // V scale of this key
                 s2 = sc | (sc << 16);
             }
-#pragma unroll 4
-            for (int cc = 0; cc < 8; ++cc) {   // 16-byte code chunk
-                const uint4 w = *reinterpret_cast<const uint4 *>(codes + swz(row, cc));
+            // all eight 16-byte code chunks of the row are loaded before any is
+            // converted: one shared-memory round trip per tile, not eight
+            uint4 wv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (i < nch)
+                    wv[i] = *reinterpret_cast<const uint4 *>(codes + swz(row, c0 + i));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                if (i >= nch)
+                    break;
+                const int cc = c0 + i;   // 16-byte code chunk
+                const uint4 w = wv[i];
                 uint32_t hv[8];
                 cvt4<KVT>(w.x, hv[0], hv[1]);
                 cvt4<KVT>(w.y, hv[2], hv[3]);
@@ -376,7 +391,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     make_uint4(hv[4], hv[5], hv[6], hv[7]);
             }
             if constexpr (KVT == kKvInt8) {
-                if (!isv) {   // per-key score factor: softmax scale * log2(e) * K scale
+                if (!isv && c0 == 0) {   // per-key score factor: softmax scale * log2(e) * K scale
                     float *ksf = reinterpret_cast<float *>(smem + kOffKsf) + bj * 64;
                     ksf[row] = live ? kfac * __half2float(__ushort_as_half(scl[row])) : 0.0f;
                 }
