@@ -20,8 +20,11 @@
 //   warp 2      TMA producer: one 2-D tensor copy per cache block and head
 //               into a 3-stage code ring; block ids come from a register window.
 //   warp 3      allocates all 512 TMEM columns (per tile: S/P 64, O 128, Q 64)
-//               and issues every MMA from one thread, ping-ponging between the
-//               tiles: O_A += P_A V, S_A = Q_A K_next, then the same for B.
+//               and issues every MMA: the whole warp runs the loop on
+//               warp-uniform values and an elected lane issues each tcgen05
+//               instruction.  It serves whichever tile has its P ready
+//               (O += P V, then S = Q K_next in the same columns), sleeping
+//               with a bounded mbarrier wait on the tile that is due.
 //               Completion is signalled with tcgen05.commit on mbarriers.
 //   warps 4-7   softmax for tile A, warps 8-11 softmax for tile B: thread i of
 //               a group owns row i (TMEM lane i): it stores its Q row in TMEM,

@@ -1,6 +1,6 @@
 // 5th-generation tensor core (tcgen05) and tensor-memory helpers for sm_100a:
-// TMEM allocation, shared-memory matrix descriptors, single-thread MMA issue
-// with mbarrier commit, and TMEM <-> register moves.  Thin PTX wrappers.
+// TMEM allocation, shared-memory matrix descriptors, MMA issue by an elected
+// lane with mbarrier commit, and TMEM <-> register moves.  Thin PTX wrappers.
 #pragma once
 
 #include "common.cuh"
@@ -67,48 +67,14 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_maj
            | ((uint32_t)(M >> 4) << 24);
 }
 
-// D[tmem] = A * B (+ D if accumulate), one thread issues.
-__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// D[tmem] = A[tmem] * B (+ D if accumulate): A read from tensor memory
-// (row m in lane m, two consecutive fp16 k values per 32-bit column).
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // Warp-wide forms: the whole (converged) warp executes the call with the same
 // operands and one lane, chosen by elect.sync, issues the instruction.  The
 // operands are then warp-uniform values the compiler can keep in uniform
 // registers, instead of values computed inside a single-lane branch.
-__device__ __forceinline__ void mma_f16_ss_elect(uint32_t d_tmem, uint64_t a_desc,
-                                                 uint64_t b_desc, uint32_t idesc,
-                                                 uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 
+// D[tmem] = A[tmem] * B (+ D if accumulate): A read from tensor memory (row m
+// in lane m, two consecutive fp16 k values per 32-bit column), B from a
+// shared-memory descriptor.
 __device__ __forceinline__ void mma_f16_ts_elect(uint32_t d_tmem, uint32_t a_tmem,
                                                  uint64_t b_desc, uint32_t idesc,
                                                  uint32_t accumulate)
@@ -122,22 +88,14 @@ __device__ __forceinline__ void mma_f16_ts_elect(uint32_t d_tmem, uint32_t a_tme
         : "memory");
 }
 
+// The mbarrier gets one arrival when every tcgen05 operation the electing
+// thread issued so far has completed.
 __device__ __forceinline__ void mma_commit_elect(uint64_t *bar)
 {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"
         "elect.sync _|e, 0xffffffff;\n\t"
         "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
-
-// The mbarrier gets one arrival when every tcgen05 operation issued so far by
-// this thread has completed.
-__device__ __forceinline__ void mma_commit(uint64_t *bar)
-{
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             smem_u32(bar))
         : "memory");
 }
