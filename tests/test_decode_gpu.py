@@ -33,6 +33,11 @@ CASES = [
     (INT8, 16, 2, [3000, 40000, 5], 2, 16),
     # more than 32 sequences: the slot map is scanned in several warp chunks
     (FP8, 8, 2, [(i * 977) % 3001 + 1 for i in range(40)], 1, 16),
+    # more than 16 rows per KV head: the tcgen05 kernel, every block size
+    (FP8, 16, 2, [1000, 333], 3, 32),       # 24 rows
+    (INT8, 8, 1, [2000, 77], 4, 64),        # 32 rows
+    (FP8, 16, 2, [900], 16, 16),            # 128 rows: one full tile
+    (FP8, 32, 2, [500], 16, 16),            # 256 rows: past the tile, mma.sync row groups
 ]
 
 
