@@ -149,3 +149,37 @@ def test_prefill_argument_checks(lib):
 
 def test_device_status_rejects_null(lib):
     assert lib.pkvq_device_status(None, 0) == INVALID
+
+
+# ---- decode plan: routing and workspace size (host only; on a machine
+# without a GPU the library assumes 148 SMs) ----
+
+def _ws(lib, batch, q_len, hq, hkv, max_ctx):
+    c = _cache(num_kv_heads=hkv)
+    return lib.pkvq_decode_workspace_bytes(batch, q_len, hq, max_ctx, ctypes.byref(c))
+
+
+def test_verify_rows_take_the_tensor_core_plan(lib, monkeypatch):
+    # 5 tokens x G = 8 -> 40 rows per KV head (17..128): one CTA for all rows,
+    # one CTA per SM, C = max(B, SMs / Hkv) slots per KV head
+    monkeypatch.delenv("PKVQ_DECODE_CTAS_PER_SM", raising=False)
+    sms, hkv, rows, batch = 148, 4, 40, 6
+    C = max(batch, sms // hkv)
+    assert _ws(lib, batch, 5, 32, hkv, 524288) == hkv * C * rows * (128 + 2) * 4
+
+
+def test_row_counts_past_one_tile_use_row_groups(lib, monkeypatch):
+    # 16 tokens x G = 16 = 256 rows: past 128, the mma.sync kernel in groups of
+    # 16 rows; the workspace holds one 16-row partial per slot and row group
+    monkeypatch.setenv("PKVQ_DECODE_CTAS_PER_SM", "2")
+    sms, hkv, batch = 148, 2, 1
+    groups = 256 // 16
+    units = hkv * groups
+    C = max(batch, 2 * sms // units)
+    assert _ws(lib, batch, 16, 32, hkv, 65536) == units * C * 16 * (128 + 2) * 4
+
+
+def test_one_slot_per_sequence_needs_no_workspace(lib, monkeypatch):
+    # more sequences than the GPU has slots for: every sequence is one split
+    monkeypatch.setenv("PKVQ_DECODE_CTAS_PER_SM", "1")
+    assert _ws(lib, 4096, 1, 32, 4, 32768) == 0
