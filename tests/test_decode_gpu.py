@@ -75,6 +75,22 @@ def test_decode_empty_context_and_q_len_beyond_context():
                  vmax=row_vmax(case, oc))
 
 
+def test_decode_tensor_core_path_empty_context_and_q_len_beyond_context():
+    # 5 tokens x G = 4 = 20 rows: the tcgen05 kernel.  Context 0 -> zeros /
+    # -inf; q_len 5 over context 3 -> the first two rows see nothing.
+    case = _case(FP8, 8, 2, [0, 3, 40], 5, 16, seed=5)
+    case.spec.context_lens = [0, 3, 40]
+    cache = gpu_cache(case)
+    oc = oracle_cache(case)
+    out, lse = run_gpu(case, cache)
+    ref, ref_lse = run_oracle(case, oc)
+    assert np.all(out[:5].numpy() == 0)
+    assert np.all(np.isneginf(lse[:5].numpy()))
+    assert np.all(out[5:7].numpy() == 0) and np.all(np.isneginf(lse[5:7].numpy()))
+    assert_close(out, ref, lse, ref_lse, what="empty rows, tcgen05 decode",
+                 vmax=row_vmax(case, oc))
+
+
 def test_decode_max_in_last_tile_and_large_logits():
     case = _case(FP8, 8, 2, [3000, 1500], 1, 16, seed=5)
     # a key at the very end of each context that aligns with every query:

@@ -22,6 +22,8 @@ CASES = [
     (FP8, 4, 2, [1, 2, 3], [1, 2, 3], 16),         # tiny sequences
     (FP8, 12, 2, [260], [130], 16),                # G = 6: 128 % 6 != 0
     (INT8, 32, 4, [2500], [1024], 16),
+    (FP8, 16, 2, [700], [300], 64),                # FP8 with 64-token blocks
+    (FP8, 8, 2, [96, 1000], [96, 33], 32),         # FP8 with 32-token blocks
 ]
 
 
