@@ -48,11 +48,7 @@ constexpr float kLn2 = 0.693147180559945309f;
 
 template <int BS>
 struct DecodeCfg {
-#ifdef PKVQ_DECODE_STAGES
-    static constexpr int kStages = BS == 16 ? PKVQ_DECODE_STAGES : (BS == 32 ? 3 : 2);
-#else
     static constexpr int kStages = BS == 16 ? 4 : (BS == 32 ? 3 : 2);
-#endif
     static constexpr int kUnroll = BS == 16 ? 2 : 1;   // cache blocks per loop iteration
     static constexpr int kTileBytes = BS * 128;
     static constexpr int kStageBytes = 2 * kTileBytes;
