@@ -198,8 +198,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     if (warp == kWarpTma) {
         // ------------------------------------------------ TMA producer --
         const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq + blk_begin;
-        int win0 = lane < nblk ? __ldg(bt + lane) : 0;
-        int win1 = 32 + lane < nblk ? __ldg(bt + 32 + lane) : 0;
+        // every index stays inside the table row, even for a context longer
+        // than the row can address (a caller error: those keys read block 0)
+        const int nwin = min(nblk, p.max_blocks_per_seq - blk_begin);
+        int win0 = lane < nwin ? __ldg(bt + lane) : 0;
+        int win1 = 32 + lane < nwin ? __ldg(bt + 32 + lane) : 0;
         int wbase = 0;
         int issued = 0;
         for (int j = 0; j < ntiles; ++j) {
@@ -250,7 +253,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             if (blk0 + kBPT >= wbase + 32) {
                 wbase += 32;
                 win0 = win1;
-                win1 = wbase + 32 + lane < nblk ? __ldg(bt + wbase + 32 + lane) : 0;
+                win1 = wbase + 32 + lane < nwin ? __ldg(bt + wbase + 32 + lane) : 0;
             }
         }
         // copies this CTA issued must land before it exits (bounded wait)

@@ -206,7 +206,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             prefetch_tmap(&vmap);
         }
         const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq;
-        const int nblk_used = min(nblk_seq, ntiles * kBPT);
+        // every index stays inside the table row, even for a context longer
+        // than the row can address (a caller error: those keys read block 0)
+        const int nblk_used = min(min(nblk_seq, ntiles * kBPT), p.max_blocks_per_seq);
         int win0 = lane < nblk_used ? __ldg(bt + lane) : 0;
         int win1 = 32 + lane < nblk_used ? __ldg(bt + 32 + lane) : 0;
         int wbase = 0;
