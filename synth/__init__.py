@@ -26,7 +26,16 @@ import torch
 
 FP8_E4M3 = 0
 INT8 = 1
+FP8_E5M2 = 2
+FP16 = 3
 E4M3_MAX = 448.0
+E5M2_MAX = 57344.0
+FP8_MAX = {FP8_E4M3: E4M3_MAX, FP8_E5M2: E5M2_MAX}
+
+
+def elem_bytes(kv_dtype: int) -> int:
+    """Bytes per stored cache element."""
+    return 2 if kv_dtype == FP16 else 1
 
 
 @dataclass
@@ -43,6 +52,8 @@ class CaseSpec:
     outlier_frac: float = 0.0    # fraction of (head, d) channels scaled x8
     seed: int = 0
     name: str = ""
+    scale_per_layer: bool = False  # FP8: one K and one V scale for all heads
+    window: int = 0              # > 0: sliding window of that many keys
 
 
 @dataclass
@@ -55,7 +66,7 @@ class Case:
     block_table: torch.Tensor    # int32 [B][max_blocks]
     context_lens: torch.Tensor   # int32 [B]
     cu_seqlens_q: torch.Tensor   # int32 [B+1]
-    k_scale: Optional[torch.Tensor]  # fp32 [Hkv] (FP8 only)
+    k_scale: Optional[torch.Tensor]  # fp32 [Hkv], or [1] per layer (FP8 only)
     v_scale: Optional[torch.Tensor]
     num_blocks: int
     softmax_scale: float
@@ -89,10 +100,17 @@ def _outliers(gen: torch.Generator, t: torch.Tensor, frac: float) -> None:
     flat[:, ch] = (flat[:, ch].float() * 8.0).to(torch.float16)
 
 
-def per_head_absmax_scale(t: torch.Tensor) -> torch.Tensor:
-    """Static calibration: fp32 absmax over tokens and d, per KV head, / 448."""
+def per_head_absmax_scale(t: torch.Tensor, fmax: float = E4M3_MAX) -> torch.Tensor:
+    """Static calibration: fp32 absmax over tokens and d, per KV head, / the
+    format's largest finite value (448 for E4M3, 57344 for E5M2)."""
     amax = t.abs().amax(dim=(0, 2)).float()
-    return amax / torch.tensor(E4M3_MAX, dtype=torch.float32)
+    return amax / torch.tensor(fmax, dtype=torch.float32)
+
+
+def per_layer_absmax_scale(t: torch.Tensor, fmax: float = E4M3_MAX) -> torch.Tensor:
+    """One scale for all heads: fp32 absmax over everything / fmax, shape [1]."""
+    amax = t.abs().amax().float().reshape(1)
+    return amax / torch.tensor(fmax, dtype=torch.float32)
 
 
 def make_case(spec: CaseSpec) -> Case:
@@ -128,9 +146,12 @@ def make_case(spec: CaseSpec) -> Case:
         offs.append(offs[-1] + c)
     cu = torch.zeros(B + 1, dtype=torch.int32)
     cu[1:] = torch.cumsum(torch.tensor(spec.q_lens, dtype=torch.int32), 0)
-    if spec.kv_dtype == FP8_E4M3:
-        k_scale = per_head_absmax_scale(k) if total_tok else torch.ones(Hkv)
-        v_scale = per_head_absmax_scale(v) if total_tok else torch.ones(Hkv)
+    if spec.kv_dtype in FP8_MAX:
+        fmax = FP8_MAX[spec.kv_dtype]
+        cal = per_layer_absmax_scale if spec.scale_per_layer else per_head_absmax_scale
+        n = 1 if spec.scale_per_layer else Hkv
+        k_scale = cal(k, fmax) if total_tok else torch.ones(n)
+        v_scale = cal(v, fmax) if total_tok else torch.ones(n)
     else:
         k_scale = v_scale = None
     softmax_scale = float(torch.tensor(1.0 / math.sqrt(D), dtype=torch.float32))
@@ -167,12 +188,54 @@ def workload(n: int, seed: int = 0) -> CaseSpec:
 
 def kv_read_bytes(spec: CaseSpec) -> int:
     """Algorithmic KV bytes one attention pass reads: every cached token's K
-    and V codes for every KV head, plus the INT8 fp16 per-token scales."""
+    and V elements for every KV head, plus the INT8 fp16 per-token scales."""
     tok = sum(spec.context_lens)
-    per_tok = 2 * spec.num_kv_heads * spec.head_dim
+    per_tok = 2 * spec.num_kv_heads * spec.head_dim * elem_bytes(spec.kv_dtype)
     if spec.kv_dtype == INT8:
         per_tok += 2 * spec.num_kv_heads * 2
     return tok * per_tok
+
+
+# ------------------------------------------------- sequence-sharded layout --
+
+@dataclass
+class Shard:
+    """The keys one rank holds when a batch's cached blocks are dealt out
+    over `world` ranks, block j of every sequence to rank j % world (the
+    decode-context-parallel layout).  Keys keep their order: local key i of
+    sequence s is in local block i // bs."""
+    block_table: torch.Tensor    # int32 [B][max local blocks] (physical ids)
+    context_lens: torch.Tensor   # int32 [B]: keys this rank holds
+    query_pos: torch.Tensor      # int32 [total_q]: each query's position in
+                                 # local key coordinates (last visible local key)
+
+
+def dcp_shard(case: Case, world: int, rank: int) -> Shard:
+    """Rank `rank`'s share of the case's blocks and the local positions of
+    its queries (how many local keys precede or equal each query's global
+    position, minus one)."""
+    s = case.spec
+    bs = s.block_size
+    B = len(s.context_lens)
+    tables, lens, qpos = [], [], []
+    for b, (c, ql) in enumerate(zip(s.context_lens, s.q_lens)):
+        nblk = (c + bs - 1) // bs
+        mine = [j for j in range(nblk) if j % world == rank]
+        tables.append([int(case.block_table[b, j]) for j in mine])
+        # global positions of the local keys, in order
+        gpos = [j * bs + o for j in mine for o in range(bs) if j * bs + o < c]
+        lens.append(len(gpos))
+        g = torch.tensor(gpos, dtype=torch.int64)
+        for t in range(ql):
+            p = c - ql + t
+            qpos.append(int((g <= p).sum()) - 1)
+    width = max(1, max((len(t) for t in tables), default=1))
+    bt = torch.zeros((B, width), dtype=torch.int32)
+    for b, t in enumerate(tables):
+        if t:
+            bt[b, :len(t)] = torch.tensor(t, dtype=torch.int32)
+    return Shard(bt, torch.tensor(lens, dtype=torch.int32),
+                 torch.tensor(qpos, dtype=torch.int32))
 
 
 def useful_flops(spec: CaseSpec) -> int:

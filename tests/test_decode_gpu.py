@@ -8,8 +8,8 @@ import torch
 
 import paged_quantized_kv_quant_b200 as pk
 import synth
-from pkvq_testutil import (assert_close, assert_codes_equal, gpu_cache, oracle_cache, row_vmax,
-                           run_gpu, run_oracle)
+from pkvq_testutil import (assert_close, assert_codes_equal, assert_matches_oracle, gpu_cache,
+                           oracle_cache, run_gpu, run_oracle)
 
 pytestmark = pytest.mark.gpu
 
@@ -47,16 +47,17 @@ def _case(dtype, Hq, Hkv, ctx, ql, bs, seed=0, **kw):
     return synth.make_case(spec)
 
 
+@pytest.mark.parametrize("outliers", [0.0, 0.01])
 @pytest.mark.parametrize("dtype,Hq,Hkv,ctx,ql,bs", CASES)
-def test_decode_matches_oracle(dtype, Hq, Hkv, ctx, ql, bs):
-    case = _case(dtype, Hq, Hkv, ctx, ql, bs, seed=21, outlier_frac=0.01)
+def test_decode_matches_oracle(dtype, Hq, Hkv, ctx, ql, bs, outliers):
+    case = _case(dtype, Hq, Hkv, ctx, ql, bs, seed=21, outlier_frac=outliers)
     cache = gpu_cache(case)
     oc = oracle_cache(case)
     assert_codes_equal(cache, oc, case)
     out, lse = run_gpu(case, cache)
     ref, ref_lse = run_oracle(case, oc)
-    assert_close(out, ref, lse, ref_lse, what=f"decode {dtype} {Hq}/{Hkv} {ctx} q{ql} bs{bs}",
-                 vmax=row_vmax(case, oc))
+    assert_matches_oracle(case, oc, out, lse, ref, ref_lse,
+                          what=f"decode {dtype} {Hq}/{Hkv} {ctx} q{ql} bs{bs} x8:{outliers}")
     assert pk.device_status() == 0
 
 
@@ -71,8 +72,7 @@ def test_decode_empty_context_and_q_len_beyond_context():
     assert np.all(out[:3].numpy() == 0)
     assert np.all(np.isneginf(lse[:3].numpy()))
     assert np.all(out[3].numpy() == 0) and np.all(np.isneginf(lse[3].numpy()))
-    assert_close(out, ref, lse, ref_lse, what="empty rows",
-                 vmax=row_vmax(case, oc))
+    assert_matches_oracle(case, oc, out, lse, ref, ref_lse, what="empty rows")
 
 
 def test_decode_tensor_core_path_empty_context_and_q_len_beyond_context():
@@ -87,8 +87,7 @@ def test_decode_tensor_core_path_empty_context_and_q_len_beyond_context():
     assert np.all(out[:5].numpy() == 0)
     assert np.all(np.isneginf(lse[:5].numpy()))
     assert np.all(out[5:7].numpy() == 0) and np.all(np.isneginf(lse[5:7].numpy()))
-    assert_close(out, ref, lse, ref_lse, what="empty rows, tcgen05 decode",
-                 vmax=row_vmax(case, oc))
+    assert_matches_oracle(case, oc, out, lse, ref, ref_lse, what="empty rows, tcgen05 decode")
 
 
 def test_decode_max_in_last_tile_and_large_logits():
@@ -104,8 +103,7 @@ def test_decode_max_in_last_tile_and_large_logits():
     oc = oracle_cache(case)
     out, lse = run_gpu(case, cache)
     ref, ref_lse = run_oracle(case, oc)
-    assert_close(out, ref, lse, ref_lse, what="peaked",
-                 vmax=row_vmax(case, oc))
+    assert_matches_oracle(case, oc, out, lse, ref, ref_lse, what="peaked")
 
 
 def test_decode_uniform_logits_mean_of_values():
@@ -115,8 +113,7 @@ def test_decode_uniform_logits_mean_of_values():
     oc = oracle_cache(case)
     out, lse = run_gpu(case, cache)
     ref, ref_lse = run_oracle(case, oc)
-    assert_close(out, ref, lse, ref_lse, what="uniform",
-                 vmax=row_vmax(case, oc))
+    assert_matches_oracle(case, oc, out, lse, ref, ref_lse, what="uniform")
     assert np.allclose(lse.numpy(), np.log(513), atol=1e-4)
 
 
@@ -151,8 +148,7 @@ def test_decode_causal_append_within_tolerance():
         case.context_lens = torch.tensor([c], dtype=torch.int32)
         out, lse = run_gpu(case, cache)
         ref, ref_lse = run_oracle(case, oc)
-        assert_close(out, ref, lse, ref_lse, what=f"ctx {c}",
-                 vmax=row_vmax(case, oc))
+        assert_matches_oracle(case, oc, out, lse, ref, ref_lse, what=f"ctx {c}")
 
 
 def test_decode_workspace_too_small_is_rejected():

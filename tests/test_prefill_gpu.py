@@ -6,7 +6,7 @@ import torch
 
 import paged_quantized_kv_quant_b200 as pk
 import synth
-from pkvq_testutil import assert_close, gpu_cache, oracle_cache, row_vmax, run_gpu, run_oracle
+from pkvq_testutil import assert_matches_oracle, gpu_cache, oracle_cache, run_gpu, run_oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -27,17 +27,17 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("outliers", [0.0, 0.01])
 @pytest.mark.parametrize("dtype,Hq,Hkv,ctx,ql,bs", CASES)
-def test_prefill_matches_oracle(dtype, Hq, Hkv, ctx, ql, bs):
+def test_prefill_matches_oracle(dtype, Hq, Hkv, ctx, ql, bs, outliers):
     spec = synth.CaseSpec("prefill", dtype, Hq, Hkv, list(ctx), list(ql), block_size=bs,
-                          seed=31, outlier_frac=0.01)
+                          seed=31, outlier_frac=outliers)
     case = synth.make_case(spec)
     cache = gpu_cache(case)
     oc = oracle_cache(case)
     out, lse = run_gpu(case, cache)
     ref, ref_lse = run_oracle(case, oc)
-    assert_close(out, ref, lse, ref_lse, what=f"prefill {dtype} {Hq}/{Hkv} {ctx} {ql} bs{bs}",
-                 vmax=row_vmax(case, oc))
+    assert_matches_oracle(case, oc, out, lse, ref, ref_lse, what=f"prefill {dtype} {Hq}/{Hkv} {ctx} {ql} bs{bs}")
     assert pk.device_status() == 0
 
 
@@ -66,8 +66,7 @@ def test_prefill_large_logits_and_max_on_diagonal():
     oc = oracle_cache(case)
     out, lse = run_gpu(case, cache)
     ref, ref_lse = run_oracle(case, oc)
-    assert_close(out, ref, lse, ref_lse, what="diagonal max",
-                 vmax=row_vmax(case, oc))
+    assert_matches_oracle(case, oc, out, lse, ref, ref_lse, what="diagonal max")
 
 
 def test_prefill_matches_decode_on_the_last_token():
