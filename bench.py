@@ -7,15 +7,20 @@ with per-KV-head scales, 1% outlier channels x8): write + quantize the step's
 new token into the paged cache (pkvq_kv_write_quant), then attend over the
 whole cache (pkvq_paged_attn_decode: split kernel + merge kernel).  The metric
 is KV-read GB/s: the K and V code bytes one step must read (268,435,456 B per
-GPU) divided by the step time.  Causal prefill TFLOP/s (8,192-token prefill,
-same heads) is reported beside it under "secondary".
+GPU) divided by the step time.
+
+The other four named workloads are measured in the same run under
+"secondary", each against its own roofline and beside the FP64 oracle timed
+on the host cores: the 1 x 1K decode (latency), the 8K causal prefill and the
+8K chunk over a 120K prefix (useful TFLOP/s against the measured dense fp16 /
+bf16 tensor peak), the 2 x 512K + 4 x 256K INT8 verify decode (KV GB/s
+against HBM), and the KV writes of the two prefills.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pkvq|reference]
-    python bench.py --only decode|prefill [--steps K] [--warmup W]
+    python bench.py --only decode|prefill [--workload n] [--steps K] [--warmup W]
 
---only runs nothing but W + K calls of one kernel path on its workload (the
-decode call on the batch-8 x 32K cache, or the 8K causal prefill) and prints
-their average time: the command the ncu captures are taken with.
+--only runs nothing but W + K calls of one kernel path on its workload and
+prints their average time: the command the ncu captures are taken with.
 
 Under torchrun every rank runs the same batch on its own GPU (no collective on
 the data path: weak scaling); the time is the max over ranks.  The reference
@@ -56,6 +61,7 @@ REFERENCE_BUDGET_S = 120.0
 E2E_GRAPH_STEPS = 8
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+MIN_TIMED_S = 0.2          # every per-kernel number: at least this much replay time
 
 
 def parse():
@@ -66,10 +72,14 @@ def parse():
     ap.add_argument("--impl", choices=["pkvq", "reference"], default="pkvq")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip every secondary workload")
     ap.add_argument("--only", choices=["decode", "prefill"], default=None)
     ap.add_argument("--workload", type=int, default=None,
                     help="with --only: the named workload to run (decode 1, 2, 5; prefill 3, 4)")
+    ap.add_argument("--ctx-div", type=int, default=1,
+                    help="with --only decode: divide every context length by this (a smaller "
+                         "case of the same shape, e.g. for a profiler capture)")
     return ap.parse_args()
 
 
@@ -99,6 +109,8 @@ class ClockSampler:
         self.period = period_s
         self.ok = False
         self.max_mhz = None
+        self.active = threading.Event()   # samples are taken only while set
+        self.active.set()
         try:
             import pynvml
             pynvml.nvmlInit()
@@ -123,8 +135,15 @@ class ClockSampler:
 
     def _run(self):
         while not self._stop.is_set():
-            self._sample()
+            if self.active.is_set():
+                self._sample()
             time.sleep(self.period)
+
+    def pause(self):
+        self.active.clear()
+
+    def resume(self):
+        self.active.set()
 
     def __enter__(self):
         if self.ok:
@@ -136,7 +155,6 @@ class ClockSampler:
         if self._t:
             self._stop.set()
             self._t.join()
-            self._sample()
 
     def summary(self):
         if not self.samples:
@@ -152,31 +170,83 @@ def _bits16(t):
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def _oracle_cache(case):
+def _oracle_cache(case, only_seqs=None):
+    """The oracle's own copy of the case's cache (quantized by the oracle);
+    only_seqs: write just those sequences' tokens (a bounded sample)."""
     import oracle
     s = case.spec
     oc = oracle.Cache(s.kv_dtype, case.num_blocks, s.block_size, s.num_kv_heads, s.head_dim,
                       None if case.k_scale is None else case.k_scale.numpy(),
-                      None if case.v_scale is None else case.v_scale.numpy())
-    oc.write(_bits16(case.k), _bits16(case.v), case.slot_mapping.numpy())
+                      None if case.v_scale is None else case.v_scale.numpy(),
+                      scale_per_layer=s.scale_per_layer)
+    if only_seqs is None:
+        oc.write(_bits16(case.k), _bits16(case.v), case.slot_mapping.numpy())
+    else:
+        for b in only_seqs:
+            lo, hi = int(case.token_offsets[b]), int(case.token_offsets[b + 1])
+            oc.write(_bits16(case.k[lo:hi]), _bits16(case.v[lo:hi]),
+                     case.slot_mapping[lo:hi].numpy())
     return oc
 
 
-def _oracle_rows(oc, case, rows):
-    """One oracle pass over the given (sequence, query head) rows; seconds, threads."""
+def _oracle_rows(oc, case, rows, nthreads=0):
+    """One oracle pass over the given (query token, head) rows; seconds, threads."""
     import oracle
     t0 = time.perf_counter()
     _, _, used = oracle.paged_attention(oc, _bits16(case.q), case.cu_seqlens_q.numpy(),
                                         case.context_lens.numpy(), case.block_table.numpy(),
                                         case.softmax_scale,
-                                        rows=np.asarray(rows, np.int32).reshape(-1, 2))
+                                        rows=np.asarray(rows, np.int32).reshape(-1, 2),
+                                        nthreads=nthreads)
     return time.perf_counter() - t0, used
 
 
 def _row_bytes(spec) -> float:
-    """Algorithmic KV bytes per (sequence, query head) row: a 1/Hq share of
-    its sequence's KV bytes (the G rows of a KV head read the same codes)."""
+    """Algorithmic KV bytes per (sequence, query head) row of a q_len-1 decode
+    with equal lengths: a 1/Hq share of its sequence's KV bytes (the G rows
+    of a KV head read the same codes)."""
     return synth.kv_read_bytes(spec) / len(spec.context_lens) / spec.num_q_heads
+
+
+def _row_work(case, rows, unit: str) -> float:
+    """Algorithmic work of the given (query token, head) rows: their share of
+    the KV bytes (decode: a row reads 1 / (Hq * q_len) of its sequence's
+    bytes) or their useful flops (4 * D per visible key)."""
+    s = case.spec
+    cu = case.cu_seqlens_q.numpy()
+    seq = np.searchsorted(cu, np.asarray(rows)[:, 0], side="right") - 1
+    tot = 0.0
+    per_tok = synth.kv_read_bytes(synth.CaseSpec(s.kind, s.kv_dtype, s.num_q_heads,
+                                                 s.num_kv_heads, [1], [1]))
+    for (i, _), b in zip(rows, seq):
+        c, ql = s.context_lens[b], s.q_lens[b]
+        if unit == "GB/s":
+            tot += c * per_tok / (s.num_q_heads * ql)
+        else:
+            tot += 4 * s.head_dim * max(0, c - ql + (i - cu[b]) + 1)
+    return tot
+
+
+def oracle_rate(case, oc, rows, unit: str, nthreads: int = 0, min_seconds: float = 3.0,
+                max_passes: int = 50):
+    """The FP64 oracle on `rows`, repeated until about min_seconds: returns
+    (value in `unit`, seconds, threads, passes)."""
+    total, passes, used = 0.0, 0, 0
+    while passes < max_passes and (passes == 0 or total < min_seconds):
+        dt, used = _oracle_rows(oc, case, rows, nthreads)
+        total += dt
+        passes += 1
+    work = _row_work(case, rows, unit) * passes
+    scale = 1e9 if unit == "GB/s" else 1e12
+    return work / total / scale, total, used, passes
+
+
+def cpu_entry(case, oc, rows, unit, what, nthreads=0, min_seconds=3.0):
+    v, dt, used, passes = oracle_rate(case, oc, rows, unit, nthreads, min_seconds)
+    return {"value": v, "unit": unit, "cores": used, "kind": "oracle",
+            "sample": f"{what}: {len(rows)} (token, head) rows x {passes} passes, FP64 oracle, "
+                      f"{dt:.1f} s; value = their share of the workload's "
+                      f"{'KV bytes' if unit == 'GB/s' else 'useful flops'} / time"}
 
 
 def oracle_decode_sample(case, min_seconds: float = 10.0, max_passes: int = 4):
@@ -237,20 +307,33 @@ def run_reference(args, rank: int):
 
 # -------------------------------------------------------------- GPU arm --
 
+def new_cache(pk, case, device):
+    s = case.spec
+    return pk.PagedKVCache.allocate(s.kv_dtype, case.num_blocks, s.block_size, s.num_kv_heads,
+                                    s.head_dim, device=device, k_scale=case.k_scale,
+                                    v_scale=case.v_scale, scale_per_layer=s.scale_per_layer)
+
+
+def write_all(pk, cache, case, device, chunk_tokens: int = 1 << 20):
+    """Writes every cached token of the case through kv_write_quant (in chunks,
+    so that the fp16 sources never all sit on the device)."""
+    T = case.k.shape[0]
+    for lo in range(0, T, chunk_tokens):
+        hi = min(T, lo + chunk_tokens)
+        pk.kv_write_quant(cache, case.k[lo:hi].to(device), case.v[lo:hi].to(device),
+                          case.slot_mapping[lo:hi].to(device))
+    torch.cuda.synchronize()
+
+
 def build_decode(case, device, copies: int = 2):
     import paged_quantized_kv_quant_b200 as pk
     s = case.spec
     B, ql, Hq, D = len(s.context_lens), s.q_lens[0], s.num_q_heads, s.head_dim
-    k_all, v_all = case.k.to(device), case.v.to(device)
-    sm_all = case.slot_mapping.to(device)
     caches = []
-    for _ in range(copies):   # two copies: consecutive steps never share L2 lines
-        c = pk.PagedKVCache.allocate(s.kv_dtype, case.num_blocks, s.block_size,
-                                     s.num_kv_heads, D, device=device,
-                                     k_scale=case.k_scale, v_scale=case.v_scale)
-        pk.kv_write_quant(c, k_all, v_all, sm_all)
+    for _ in range(copies):   # several copies: consecutive calls never share L2 lines
+        c = new_cache(pk, case, device)
+        write_all(pk, c, case, device)
         caches.append(c)
-    del k_all, v_all, sm_all
     new = case.new_token_rows()
     inp = {
         "q": case.q.view(B, ql, Hq, D).to(device),
@@ -263,7 +346,7 @@ def build_decode(case, device, copies: int = 2):
     inp["out"] = torch.empty_like(inp["q"])
     max_ctx = max(s.context_lens)
     ws_bytes = pk.decode_workspace_bytes(caches[0], B, ql, Hq, max_ctx)
-    inp["ws"] = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+    inp["ws"] = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=device)
     return caches, inp, max_ctx, ws_bytes
 
 
@@ -282,37 +365,97 @@ def capture(fn, stream):
     return g
 
 
-def time_graph(graph, reps, stream, barrier=None):
-    """Average ms per replay over `reps` replays, bracketed by a barrier and a
-    device synchronize on both sides, CUDA events on the launching stream."""
+def time_graphs(graphs, reps, stream, barrier=None, clk=None):
+    """Average ms per replay over `reps` replays that cycle through `graphs`,
+    bracketed by a barrier and a device synchronize on both sides, CUDA events
+    on the launching stream (clock samples taken only meanwhile)."""
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     if barrier:
         barrier()
     torch.cuda.synchronize()
+    if clk:
+        clk.resume()
     with torch.cuda.stream(stream):   # replay() launches on the current stream
         e0.record(stream)
-        for _ in range(reps):
-            graph.replay()
+        for i in range(reps):
+            graphs[i % len(graphs)].replay()
         e1.record(stream)
     torch.cuda.synchronize()
+    if clk:
+        clk.pause()
     if barrier:
         barrier()
     return e0.elapsed_time(e1) / reps
 
 
-DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_b8_ctx32k_fp8_ncu.md")
-DECODE_SOURCES = ("paged_quantized_kv_quant_b200/csrc/decode.cu",
-                  "paged_quantized_kv_quant_b200/csrc/common.cuh")
+def time_graphs_min(graphs, stream, clk=None, barrier=None, min_s=MIN_TIMED_S, warm=3):
+    """time_graphs over enough replays for at least min_s of device time."""
+    with torch.cuda.stream(stream):
+        for i in range(warm):
+            graphs[i % len(graphs)].replay()
+    probe = time_graphs(graphs, max(2, len(graphs)), stream)
+    reps = max(len(graphs) * 2, int(math.ceil(min_s * 1e3 / max(probe, 1e-4))))
+    reps = (reps + len(graphs) - 1) // len(graphs) * len(graphs)
+    return time_graphs(graphs, reps, stream, barrier, clk), reps
 
 
-def decode_sources_digest() -> str:
+def time_graph(graph, reps, stream, barrier=None):
+    return time_graphs([graph], reps, stream, barrier)
+
+
+PROFILES = {
+    "decode2": ("decode_b8_ctx32k_fp8_ncu.md",
+                ("paged_quantized_kv_quant_b200/csrc/decode.cu",
+                 "paged_quantized_kv_quant_b200/csrc/common.cuh")),
+    "decode5": ("decode_verify_q5_2x512k_4x256k_int8_ncu.md",
+                ("paged_quantized_kv_quant_b200/csrc/decode_tn.cu",
+                 "paged_quantized_kv_quant_b200/csrc/decode.cu",
+                 "paged_quantized_kv_quant_b200/csrc/split_map.cuh",
+                 "paged_quantized_kv_quant_b200/csrc/common.cuh",
+                 "paged_quantized_kv_quant_b200/csrc/tc.cuh")),
+    "prefill3": ("prefill_8k_causal_fp8_ncu.md",
+                 ("paged_quantized_kv_quant_b200/csrc/prefill_tc.cu",
+                  "paged_quantized_kv_quant_b200/csrc/common.cuh",
+                  "paged_quantized_kv_quant_b200/csrc/tc.cuh")),
+}
+DECODE_PROFILE = os.path.join(ROOT, "profiles", PROFILES["decode2"][0])
+DECODE_SOURCES = PROFILES["decode2"][1]
+
+
+def sources_digest(sources) -> str:
     import hashlib
     h = hashlib.sha256()
-    for rel in DECODE_SOURCES:
+    for rel in sources:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def decode_sources_digest() -> str:
+    return sources_digest(DECODE_SOURCES)
+
+
+def traffic_from_profile(key: str):
+    """DRAM bytes (read + write) of one call of a kernel path from its
+    committed ncu summary; None when the summary is missing or was taken on
+    other sources than the ones built now."""
+    import re
+    name, sources = PROFILES[key]
+    try:
+        with open(os.path.join(ROOT, "profiles", name)) as f:
+            text = f.read()
+    except OSError:
+        return None
+    m = re.search(r"dram_bytes_per_call:\s*([0-9]+)", text)
+    d = re.search(r"sources_digest:\s*([0-9a-f]+)", text)
+    if not m or not d or d.group(1) != sources_digest(sources):
+        return None
+    return int(m.group(1))
+
+
+def decode_traffic_from_profile():
+    return traffic_from_profile("decode2")
 
 
 def reduce_max(x: float, dist=None, device=None) -> float:
@@ -331,23 +474,6 @@ def job_throughput(world: int, bytes_per_rank: float, ms_max: float) -> float:
     return world * bytes_per_rank / (ms_max * 1e-3) / 1e9
 
 
-def decode_traffic_from_profile():
-    """DRAM bytes (read + write) of one decode call, split and merge kernels,
-    from the committed ncu summary; None when the summary is missing or was
-    taken on other decode sources than the ones built now."""
-    import re
-    try:
-        with open(DECODE_PROFILE) as f:
-            text = f.read()
-    except OSError:
-        return None
-    m = re.search(r"dram_bytes_per_call:\s*([0-9]+)", text)
-    d = re.search(r"decode_sources_digest:\s*([0-9a-f]+)", text)
-    if not m or not d or d.group(1) != decode_sources_digest():
-        return None
-    return int(m.group(1))
-
-
 def run_only(args):
     """W + K calls of one path, nothing else (for profiler captures)."""
     import paged_quantized_kv_quant_b200 as pk
@@ -357,6 +483,9 @@ def run_only(args):
     stream = torch.cuda.Stream(device=device)
     if args.only == "decode":
         spec = synth.workload(args.workload or DECODE_WORKLOAD)
+        if args.ctx_div > 1:
+            spec.context_lens = [max(spec.block_size, c // args.ctx_div) for c in spec.context_lens]
+            spec.name += f"_ctx_div{args.ctx_div}"
         case = synth.make_case(spec)
         # two cache copies alternate when they are small; one copy of a
         # cache larger than L2 already defeats it
@@ -368,10 +497,8 @@ def run_only(args):
     else:
         spec = synth.workload(args.workload or PREFILL_WORKLOAD)
         case = synth.make_case(spec)
-        c = pk.PagedKVCache.allocate(spec.kv_dtype, case.num_blocks, spec.block_size,
-                                     spec.num_kv_heads, device=device,
-                                     k_scale=case.k_scale, v_scale=case.v_scale)
-        pk.kv_write_quant(c, case.k.to(device), case.v.to(device), case.slot_mapping.to(device))
+        c = new_cache(pk, case, device)
+        write_all(pk, c, case, device)
         q = case.q.to(device)
         out = torch.empty_like(q)
         cu, bt, ctx = (case.cu_seqlens_q.to(device), case.block_table.to(device),
@@ -392,6 +519,165 @@ def run_only(args):
     torch.cuda.synchronize()
     print(json.dumps({"only": args.only, "workload": spec.name, "calls": max(1, args.steps),
                       "ms_per_call": e0.elapsed_time(e1) / max(1, args.steps)}), flush=True)
+
+
+# ------------------------------------------------------------ secondaries --
+
+def sec_decode(pk, n, device, stream, clk, hbm_peak, peak_src, copies=None):
+    """Decode workload n (1 or 5): KV GB/s of one call against HBM.  Enough
+    cache copies alternate that the inputs exceed L2."""
+    spec = synth.workload(n)
+    case = synth.make_case(spec)
+    kvb = synth.kv_read_bytes(spec)
+    if copies is None:
+        copies = max(1, int(math.ceil(160e6 / kvb)))   # > 126 MB of L2 in total
+    caches, inp, max_ctx, _ = build_decode(case, device, copies=copies)
+    sc = case.softmax_scale
+    with torch.cuda.stream(stream):
+        for c in caches:
+            decode_step(pk, c, inp, max_ctx, sc, write=False)
+    torch.cuda.synchronize()
+    graphs = [capture(lambda c=c: decode_step(pk, c, inp, max_ctx, sc, write=False), stream)
+              for c in caches]
+    ms, reps = time_graphs_min(graphs, stream, clk)
+    gbs = kvb / (ms * 1e-3) / 1e9
+    entry = {"workload": spec.name, "metric": "decode KV-read GB/s", "value": gbs,
+             "unit": "GB/s", "us_per_call": ms * 1e3, "timed_calls": reps,
+             "algorithmic_bytes": kvb,
+             "l2": f"{copies} cache copies alternated ({copies * kvb / 1e6:.0f} MB)",
+             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                          "frac": gbs / hbm_peak, "peak_source": peak_src,
+                          "traffic": traffic_from_profile("decode5") if n == 5 else None}}
+    del graphs, caches, inp
+    torch.cuda.empty_cache()
+    return entry, case
+
+
+def sec_prefill(pk, n, device, stream, clk, bf16_peak, hbm_peak, peak_src):
+    """Prefill workload n (3 or 4): useful TFLOP/s of one call against the
+    measured dense 16-bit tensor peak, and the KV write of all its tokens."""
+    spec = synth.workload(n)
+    case = synth.make_case(spec)
+    c = new_cache(pk, case, device)
+    T = case.k.shape[0]
+    kd, vd, smd = case.k.to(device), case.v.to(device), case.slot_mapping.to(device)
+    q = case.q.to(device)
+    out = torch.empty_like(q)
+    cu, bt, ctx = (case.cu_seqlens_q.to(device), case.block_table.to(device),
+                   case.context_lens.to(device))
+    mq = max(spec.q_lens)
+    sc = case.softmax_scale
+    with torch.cuda.stream(stream):
+        pk.kv_write_quant(c, kd, vd, smd)
+        pk.paged_attn_prefill(c, q, cu, bt, ctx, mq, sc, out=out)
+    torch.cuda.synchronize()
+    g_pf = capture(lambda: pk.paged_attn_prefill(c, q, cu, bt, ctx, mq, sc, out=out), stream)
+    g_wr = capture(lambda: pk.kv_write_quant(c, kd, vd, smd), stream)
+    ms_pf, reps_pf = time_graphs_min([g_pf], stream, clk)
+    ms_wr, reps_wr = time_graphs_min([g_wr], stream, clk)
+    flops = synth.useful_flops(spec)
+    tf = flops / (ms_pf * 1e-3) / 1e12
+    wbytes = T * spec.num_kv_heads * spec.head_dim * (2 * 2 + 2)   # fp16 K,V in; codes out
+    wgbs = wbytes / (ms_wr * 1e-3) / 1e9
+    entry = {"workload": spec.name, "metric": "causal prefill useful TFLOP/s", "value": tf,
+             "unit": "TFLOP/s", "ms": ms_pf, "timed_calls": reps_pf, "useful_flop": flops,
+             "frac_of_bf16_peak": tf / bf16_peak, "peak": bf16_peak, "peak_source": peak_src,
+             "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16_peak,
+                          "unit": "TFLOP/s", "frac": tf / bf16_peak, "peak_source": peak_src,
+                          "traffic": traffic_from_profile("prefill3") if n == 3 else None}}
+    wentry = {"workload": f"kv_write_quant of {spec.name} ({T} tokens)", "value": wgbs,
+              "unit": "GB/s", "ms": ms_wr, "timed_calls": reps_wr, "bytes": wbytes,
+              "frac": wgbs / hbm_peak,
+              "roofline": {"bound": "hbm", "achieved": wgbs, "peak": hbm_peak, "unit": "GB/s",
+                           "frac": wgbs / hbm_peak, "peak_source": peak_src, "traffic": None}}
+    del g_pf, g_wr, c, kd, vd, smd, q, out
+    torch.cuda.empty_cache()
+    return entry, wentry, case
+
+
+def sec_format_decode(pk, kv_dtype, device, stream, clk, hbm_peak, peak_src):
+    """The batch-8 x 32K decode with another cache format (E5M2: the same
+    bytes as E4M3; FP16: twice as many): KV GB/s of one call."""
+    base = synth.workload(DECODE_WORKLOAD)
+    name = {synth.FP8_E5M2: "e5m2", synth.FP16: "fp16"}[kv_dtype]
+    spec = synth.CaseSpec("decode", kv_dtype, base.num_q_heads, base.num_kv_heads,
+                          base.context_lens, base.q_lens, outlier_frac=base.outlier_frac,
+                          seed=base.seed, name=base.name.replace("e4m3", name))
+    case = synth.make_case(spec)
+    kvb = synth.kv_read_bytes(spec)
+    caches, inp, max_ctx, _ = build_decode(case, device, copies=2)
+    sc = case.softmax_scale
+    with torch.cuda.stream(stream):
+        for c in caches:
+            decode_step(pk, c, inp, max_ctx, sc, write=False)
+    torch.cuda.synchronize()
+    graphs = [capture(lambda c=c: decode_step(pk, c, inp, max_ctx, sc, write=False), stream)
+              for c in caches]
+    ms, reps = time_graphs_min(graphs, stream, clk)
+    gbs = kvb / (ms * 1e-3) / 1e9
+    del graphs, caches, inp
+    torch.cuda.empty_cache()
+    return {"workload": spec.name, "metric": "decode KV-read GB/s", "value": gbs, "unit": "GB/s",
+            "us_per_call": ms * 1e3, "timed_calls": reps, "algorithmic_bytes": kvb,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": gbs / hbm_peak, "peak_source": peak_src, "traffic": None}}
+
+
+def sec_block_copy(pk, device, stream, clk):
+    """KV page copies between the GPU pool and a pinned host tier (E4M3 cache of
+    the batch-8 x 32K shape, 1 GiB of blocks each way), against a plain pinned
+    copy of the same bytes measured in the same run."""
+    nb, bs, hkv = 65536, 16, 4
+    blk_bytes = 2 * hkv * bs * 128                    # K and V of one block
+    dev = pk.PagedKVCache.allocate(synth.FP8_E4M3, nb, bs, hkv, device=device,
+                                   k_scale=[1.0] * hkv, v_scale=[1.0] * hkv)
+    host = pk.PagedKVCache.allocate(synth.FP8_E4M3, nb, bs, hkv, device="cpu", pin_host=True,
+                                    k_scale=[1.0] * hkv, v_scale=[1.0] * hkv)
+    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(0)).to(torch.int32)
+    out_pairs = torch.stack([torch.arange(nb, dtype=torch.int32), perm], 1).to(device)
+    in_pairs = torch.stack([perm, torch.arange(nb, dtype=torch.int32)], 1).to(device)
+    with torch.cuda.stream(stream):
+        pk.kv_copy_blocks(host, dev, out_pairs)
+        pk.kv_copy_blocks(dev, host, in_pairs)
+    torch.cuda.synchronize()
+    g_out = capture(lambda: pk.kv_copy_blocks(host, dev, out_pairs), stream)
+    g_in = capture(lambda: pk.kv_copy_blocks(dev, host, in_pairs), stream)
+    ms_out, _ = time_graphs_min([g_out], stream, clk, min_s=0.5)
+    ms_in, _ = time_graphs_min([g_in], stream, clk, min_s=0.5)
+    # reference: one contiguous pinned copy of the same bytes each way
+    flat_d, flat_h = dev.k_cache.view(-1), host.k_cache.view(-1)
+    with torch.cuda.stream(stream):
+        flat_h.copy_(flat_d, non_blocking=True)
+    torch.cuda.synchronize()
+    g_d2h = capture(lambda: (host.k_cache.copy_(dev.k_cache, non_blocking=True),
+                             host.v_cache.copy_(dev.v_cache, non_blocking=True)), stream)
+    g_h2d = capture(lambda: (dev.k_cache.copy_(host.k_cache, non_blocking=True),
+                             dev.v_cache.copy_(host.v_cache, non_blocking=True)), stream)
+    ms_d2h, _ = time_graphs_min([g_d2h], stream, clk, min_s=0.5)
+    ms_h2d, _ = time_graphs_min([g_h2d], stream, clk, min_s=0.5)
+    total = nb * blk_bytes
+    gbs = lambda ms: total / (ms * 1e-3) / 1e9
+    del g_out, g_in, g_d2h, g_h2d, dev, host
+    torch.cuda.empty_cache()
+    return {"workload": f"kv_copy_blocks, {nb} E4M3 blocks of 16 tokens x 4 heads "
+                        f"({total >> 20} MiB) in a random order, GPU pool <-> pinned host tier",
+            "metric": "page copy GB/s", "unit": "GB/s",
+            "to_host": {"value": gbs(ms_out), "ms": ms_out,
+                        "frac_of_pinned_memcpy": ms_d2h / ms_out},
+            "to_device": {"value": gbs(ms_in), "ms": ms_in,
+                          "frac_of_pinned_memcpy": ms_h2d / ms_in},
+            "pinned_memcpy_gbs": {"d2h": gbs(ms_d2h), "h2d": gbs(ms_h2d)},
+            "roofline": {"bound": "host link", "peak": "a contiguous pinned cudaMemcpy of the "
+                                                       "same bytes, measured in this run"}}
+
+
+def prefill_sample_rows(case, n_rows, seed):
+    """Random (token, head) rows of a prefill chunk, spread over the whole chunk."""
+    rng = np.random.default_rng(seed)
+    s = case.spec
+    total = int(case.cu_seqlens_q[-1])
+    return np.stack([rng.integers(total, size=n_rows), rng.integers(s.num_q_heads, size=n_rows)],
+                    1).astype(np.int32)
 
 
 def main():
@@ -423,6 +709,10 @@ def main():
     def max_over_ranks(x: float) -> float:
         return reduce_max(x, dist, device)
 
+    clk = ClockSampler(device.index)
+    clk.pause()
+    clk.__enter__()
+
     # ---------------- decode workload ----------------
     spec = synth.workload(DECODE_WORKLOAD)
     case = synth.make_case(spec)
@@ -436,27 +726,24 @@ def main():
         for c in caches:        # warm up library state (function attributes, maps) outside capture
             decode_step(pk, c, inp, max_ctx, scale)
     torch.cuda.synchronize()
-    g_step = capture(lambda: [decode_step(pk, c, inp, max_ctx, scale) for c in caches], stream)
-    g_dec = capture(lambda: [decode_step(pk, c, inp, max_ctx, scale, write=False) for c in caches],
-                    stream)
-    g_wr = capture(lambda: [decode_step(pk, c, inp, max_ctx, scale, decode=False) for c in caches],
-                   stream)
-    reps = max(1, args.steps // 2)
-    steps = 2 * reps
-    warm = max(2, (args.warmup + 1) // 2)
+    # one graph per cache copy: consecutive steps alternate the copies
+    g_step = [capture(lambda c=c: decode_step(pk, c, inp, max_ctx, scale), stream)
+              for c in caches]
+    g_dec = [capture(lambda c=c: decode_step(pk, c, inp, max_ctx, scale, write=False), stream)
+             for c in caches]
+    g_wr = [capture(lambda c=c: decode_step(pk, c, inp, max_ctx, scale, decode=False), stream)
+            for c in caches]
+    steps = max(1, args.steps)
     with torch.cuda.stream(stream):
-        for _ in range(warm):
-            g_step.replay()
+        for i in range(max(0, args.warmup)):
+            g_step[i % 2].replay()
     torch.cuda.synchronize()
-    with ClockSampler(device.index) as clk:
-        ms_pair = time_graph(g_step, reps, stream, barrier)
-    ms_step = max_over_ranks(ms_pair / 2)
-    # per-kernel timing (same graphs, same inputs): decode call alone, write alone
-    with torch.cuda.stream(stream):
-        for _ in range(warm):
-            g_dec.replay()
-    ms_dec = max_over_ranks(time_graph(g_dec, reps, stream, barrier) / 2)
-    ms_wr = max_over_ranks(time_graph(g_wr, reps, stream, barrier) / 2)
+    ms_step = max_over_ranks(time_graphs(g_step, steps, stream, barrier, clk))
+    # per-kernel timing (same graphs, same inputs), each over >= MIN_TIMED_S
+    ms_dec, reps_dec = time_graphs_min(g_dec, stream, clk, barrier)
+    ms_dec = max_over_ranks(ms_dec)
+    ms_wr, _ = time_graphs_min(g_wr, stream, clk, barrier)
+    ms_wr = max_over_ranks(ms_wr)
     value = job_throughput(world, kv_bytes, ms_step)
     dec_gbs = kv_bytes / (ms_dec * 1e-3) / 1e9
 
@@ -531,48 +818,30 @@ def main():
     ms_e2e = max_over_ranks(time_graph(g_e2e, n_rep, stream, barrier) / E2E_GRAPH_STEPS)
     e2e_val = job_throughput(world, kv_bytes, ms_e2e)
     ok_out = bool(torch.equal(host_out[(n_e2e - 1) % 2].to(device), dev_out[(n_e2e - 1) % 2]))
+    del g_step, g_dec, g_wr, g_e2e, dev_in, dev_out
+    caches_keep = caches
+    del caches
+    torch.cuda.empty_cache()
 
-    # ---------------- secondary: causal prefill 8K ----------------
+    # ---------------- the other four workloads ----------------
     secondary = None
+    cases = {DECODE_WORKLOAD: case}
     if not args.no_prefill:
-        pspec = synth.workload(PREFILL_WORKLOAD)
-        pcase = synth.make_case(pspec)
-        pc = pk.PagedKVCache.allocate(pspec.kv_dtype, pcase.num_blocks, pspec.block_size,
-                                      pspec.num_kv_heads, device=device,
-                                      k_scale=pcase.k_scale, v_scale=pcase.v_scale)
-        pk_, pv_ = pcase.k.to(device), pcase.v.to(device)
-        psm = pcase.slot_mapping.to(device)
-        pq = pcase.q.to(device)
-        pout = torch.empty_like(pq)
-        pcu, pbt, pctx = (pcase.cu_seqlens_q.to(device), pcase.block_table.to(device),
-                          pcase.context_lens.to(device))
-        mq = max(pspec.q_lens)
-        with torch.cuda.stream(stream):
-            pk.kv_write_quant(pc, pk_, pv_, psm)
-            pk.paged_attn_prefill(pc, pq, pcu, pbt, pctx, mq, pcase.softmax_scale, out=pout)
-        torch.cuda.synchronize()
-        g_pf = capture(lambda: pk.paged_attn_prefill(pc, pq, pcu, pbt, pctx, mq,
-                                                     pcase.softmax_scale, out=pout), stream)
-        g_pw = capture(lambda: pk.kv_write_quant(pc, pk_, pv_, psm), stream)
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                g_pf.replay()
-        preps = 20
-        ms_pf = max_over_ranks(time_graph(g_pf, preps, stream, barrier))
-        ms_pw = max_over_ranks(time_graph(g_pw, preps, stream, barrier))
-        flops = synth.useful_flops(pspec)
-        wbytes = pcase.k.numel() * 2 * 2 + pcase.k.numel() * 2   # fp16 in, codes out
-        secondary = {
-            "prefill": {"workload": pspec.name, "metric": "causal prefill useful TFLOP/s",
-                        "value": flops / (ms_pf * 1e-3) / 1e12, "unit": "TFLOP/s",
-                        "ms": ms_pf, "useful_flop": flops,
-                        "frac_of_bf16_peak": flops / (ms_pf * 1e-3) / 1e12 / bf16_peak,
-                        "peak": bf16_peak, "peak_source": peak_src},
-            "kv_write_8k": {"value": wbytes / (ms_pw * 1e-3) / 1e9, "unit": "GB/s",
-                            "ms": ms_pw, "bytes": wbytes,
-                            "frac": wbytes / (ms_pw * 1e-3) / 1e9 / hbm_peak},
-        }
-        del pc, pk_, pv_
+        del caches_keep
+        torch.cuda.empty_cache()
+        secondary = {}
+        e1, cases[1] = sec_decode(pk, 1, device, stream, clk, hbm_peak, peak_src)
+        e3, w3, cases[3] = sec_prefill(pk, 3, device, stream, clk, bf16_peak, hbm_peak, peak_src)
+        e4, w4, cases[4] = sec_prefill(pk, 4, device, stream, clk, bf16_peak, hbm_peak, peak_src)
+        e5, cases[5] = sec_decode(pk, 5, device, stream, clk, hbm_peak, peak_src)
+        secondary = {"decode_1x1k": e1, "prefill": e3, "chunked_prefill": e4,
+                     "verify_decode": e5, "kv_write_8k": w3, "kv_write_131k": w4,
+                     "decode_e5m2": sec_format_decode(pk, synth.FP8_E5M2, device, stream, clk,
+                                                      hbm_peak, peak_src),
+                     "decode_fp16": sec_format_decode(pk, synth.FP16, device, stream, clk,
+                                                      hbm_peak, peak_src),
+                     "block_copy": sec_block_copy(pk, device, stream, clk)}
+    clk.__exit__()
 
     # ---------------- CPU baseline (oracle, rank 0, N = 1) ----------------
     cpu = None
@@ -581,12 +850,43 @@ def main():
         cpu = {"value": gbs, "unit": "GB/s", "cores": used, "kind": "oracle",
                "sample": f"the whole batch-8 x 32K decode (all 256 rows, 268,435,456 KV "
                          f"bytes) x {passes} passes, FP64 oracle, {dt:.1f} s"}
+        oc2 = _oracle_cache(case)
+        cpu_1core = cpu_entry(case, oc2, [[b, 0] for b in range(8)], "GB/s",
+                              "batch-8 x 32K decode, head 0 of every sequence", nthreads=1)
+        cpu["single_core"] = cpu_1core
+        del oc2
+        if secondary:
+            c1 = cases[1]
+            oc = _oracle_cache(c1)
+            rows1 = [[0, h] for h in range(c1.spec.num_q_heads)]
+            secondary["decode_1x1k"]["cpu_baseline"] = cpu_entry(
+                c1, oc, rows1, "GB/s", "the whole 1 x 1K decode")
+            secondary["decode_1x1k"]["cpu_baseline"]["single_core"] = cpu_entry(
+                c1, oc, rows1, "GB/s", "the whole 1 x 1K decode", nthreads=1)
+            c3 = cases[3]
+            oc = _oracle_cache(c3)
+            rows3 = prefill_sample_rows(c3, 256, 3)
+            secondary["prefill"]["cpu_baseline"] = cpu_entry(
+                c3, oc, rows3, "TFLOP/s", "8K causal prefill, random rows")
+            secondary["prefill"]["cpu_baseline"]["single_core"] = cpu_entry(
+                c3, oc, rows3[:16], "TFLOP/s", "8K causal prefill, random rows", nthreads=1)
+            c4 = cases[4]
+            oc = _oracle_cache(c4)
+            secondary["chunked_prefill"]["cpu_baseline"] = cpu_entry(
+                c4, oc, prefill_sample_rows(c4, 64, 4), "TFLOP/s",
+                "8K chunk over a 120K prefix, random rows")
+            c5 = cases[5]
+            oc = _oracle_cache(c5, only_seqs=[2])      # one 256K sequence of the six
+            rows5 = [[2 * 5 + t, h] for t in range(5) for h in range(0, 32, 4)]
+            secondary["verify_decode"]["cpu_baseline"] = cpu_entry(
+                c5, oc, rows5, "GB/s", "verify decode, one 256K sequence, 5 tokens x 8 heads")
+            del oc
 
     launches_per_step = 2 + (1 if plan_splits else 0)
     traffic = decode_traffic_from_profile()
     line = {
         "metric": METRIC,
-        "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": 2 * warm,
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16 (E4M3 codes dequantised to f16, f32 accumulate)",
         "data": "synthetic (seeded N(0,1), 1% channels x8)",
@@ -602,15 +902,14 @@ def main():
         "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": dec_gbs / hbm_peak, "traffic": traffic,
                      "kernel": "pkvq_paged_attn_decode (split + merge kernels)",
-                     "ms_per_launch": ms_dec, "algorithmic_bytes": kv_bytes,
-                     "peak_source": peak_src},
+                     "ms_per_launch": ms_dec, "timed_calls": reps_dec,
+                     "algorithmic_bytes": kv_bytes, "peak_source": peak_src},
         "kv_write_ms": ms_wr,
         "cpu_baseline": cpu,
         "secondary": secondary,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g_step, g_dec, g_wr, g_e2e
     if dist:
         dist.barrier()
         dist.destroy_process_group()

@@ -63,7 +63,15 @@ typedef enum {
     /* INT8 with one fp16 scale per (token, KV head), computed when the token
      * is written.  Source: "ReVolta" PyPI page, "INT8 KV" (scales computed per
      * token and head at run time, no calibration). */
-    PKVQ_KV_INT8 = 1
+    PKVQ_KV_INT8 = 1,
+    /* FP8 E5M2 (bias 15, S.11111.00 = inf, S.11111.xx = NaN, max 57344) with
+     * the same static fp32 scales as E4M3.  Source: "1Cat-LLM" README,
+     * current SM70 work list ("FP8 E4M3 / E5M2 KV storage"). */
+    PKVQ_KV_FP8_E5M2 = 2,
+    /* The fp16 values themselves, no scale (2 bytes per element).  Source:
+     * "ReVolta" PyPI page, first section ("KV formats: FP8 E4M3, FP16, and
+     * INT8"). */
+    PKVQ_KV_FP16 = 3
 } pkvq_kv_dtype;
 
 /* Describes caller-owned cache memory.  All pointers device, 16-byte aligned. */
@@ -73,12 +81,17 @@ typedef struct {
     int32_t block_size;     /* tokens per block: 16, 32 or 64 */
     int32_t num_kv_heads;
     int32_t head_dim;       /* must be 128 */
-    void *k_cache;          /* uint8 [num_blocks][num_kv_heads][block_size][head_dim] */
+    void *k_cache;          /* [num_blocks][num_kv_heads][block_size][head_dim] elements:
+                               1 byte (E4M3, E5M2, INT8) or 2 (FP16) */
     void *v_cache;
-    const float *k_scale;   /* FP8: fp32 [num_kv_heads]; INT8: NULL */
+    const float *k_scale;   /* FP8 formats: fp32 [num_kv_heads] (or [1], see
+                               scale_per_layer); INT8, FP16: unused (NULL) */
     const float *v_scale;
-    void *k_scale_tok;      /* INT8: fp16 [num_blocks][num_kv_heads][block_size]; FP8: NULL */
+    void *k_scale_tok;      /* INT8: fp16 [num_blocks][num_kv_heads][block_size]; else NULL */
     void *v_scale_tok;
+    int32_t scale_per_layer; /* FP8 formats: nonzero = k_scale and v_scale hold one value
+                                each, shared by every KV head ("ReVolta" PyPI page, "E4M3
+                                KV": one calibrated K and V scale per layer) */
 } pkvq_cache;
 
 /*
@@ -89,8 +102,10 @@ typedef struct {
  *
  * For every token i < num_tokens with slot_mapping[i] >= 0 and every KV head
  * h, writes row (slot / block_size, h, slot % block_size):
- *   FP8:  code[d] = E4M3_rn_satfinite(fp32(x[d]) / k_scale[h]) (scale 0 -> 0);
+ *   E4M3: code[d] = E4M3_rn_satfinite(fp32(x[d]) / k_scale[h]) (scale 0 -> 0);
  *         NaN keeps its sign as S.1111.111, +-inf saturates to +-448.
+ *   E5M2: the same with E5M2: NaN -> S.11111.11, +-inf saturates to +-57344.
+ *   FP16: the fp16 bits of x as given.
  *   INT8: s = fp16_rn(fp32(max_d |x[d]|) / 127);
  *         code[d] = clamp(rint(fp32(x[d]) / fp32(s)), -127, 127), s == 0 -> 0;
  *         s is stored in k_scale_tok / v_scale_tok.  Inputs must be finite.
@@ -106,9 +121,10 @@ PKVQ_API pkvq_status pkvq_kv_write_quant(const pkvq_cache *cache, const void *k,
 
 /*
  * Workspace bytes pkvq_paged_attn_decode needs for this shape on the
- * current device (split-KV partial states: fp32 O, max and sum per split).
- * Returns 0 on invalid arguments.  The same arguments give the same size and
- * the same split plan in pkvq_paged_attn_decode.
+ * current device: a leading area of arrival counters (the same size for
+ * every shape on a device) and the split-KV partial states (fp32 O, max and
+ * sum per split).  Returns 0 on invalid arguments.  The same arguments give
+ * the same size and the same split plan in pkvq_paged_attn_decode.
  */
 PKVQ_API size_t pkvq_decode_workspace_bytes(int32_t batch, int32_t q_len, int32_t num_q_heads,
                                    int32_t max_context_len, const pkvq_cache *cache);
@@ -133,12 +149,17 @@ PKVQ_API size_t pkvq_decode_workspace_bytes(int32_t batch, int32_t q_len, int32_
  *                 The kernels split each sequence's tokens over CTAs in
  *                 proportion to its own context length, read on the device.
  *   softmax_scale scores are softmax_scale * q . k_dequantized.
- *   workspace     device scratch of at least pkvq_decode_workspace_bytes();
- *                 contents need not be initialised.  Calls that overlap on
- *                 the device must not share a workspace.
+  *   workspace     device scratch of at least pkvq_decode_workspace_bytes(),
+ *                 zero-filled before its first use (e.g. cudaMemset once at
+ *                 allocation); every call leaves it ready for the next, of
+ *                 any shape.  (The last CTA of each split sequence merges it,
+ *                 found through counters that it resets.)  After a device-side
+ *                 wait timeout (pkvq_device_status bit 0) zero it again.
+ *                 Calls that overlap on the device must not share a workspace.
  * num_q_heads must be a multiple of num_kv_heads with a group of at most 16.
  * Up to 16 query rows per KV head (q_len x group) run on mma.sync tiles;
- * 17 to 128 rows run all rows of a KV head in one tcgen05 CTA.
+ * 17 to 64 rows run all rows of a KV head in one tcgen05 CTA with the keys
+ * on the tensor core's M dimension, 65 to 128 with the rows on M.
  */
 PKVQ_API pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void *q, void *out,
                                    float *lse_out, const int32_t *block_table,
@@ -160,7 +181,8 @@ PKVQ_API pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void 
  * looks up the array's device address; make that first call before any
  * stream capture.  All calls on a device share the array: calls that may
  * overlap on the device race and must be ordered by the caller.  The array
- * needs no clearing between calls.
+ * is zero when the library loads and needs no clearing between calls (each
+ * call returns its arrival counters to zero).
  */
 PKVQ_API pkvq_status pkvq_paged_attn_decode_noalloc(const pkvq_cache *cache, const void *q,
                                    void *out, float *lse_out, const int32_t *block_table,
@@ -189,6 +211,90 @@ PKVQ_API pkvq_status pkvq_paged_attn_prefill(const pkvq_cache *cache, const void
                                     int32_t max_q_len, int32_t num_q_heads,
                                     float softmax_scale, void *workspace,
                                     size_t workspace_bytes, void *stream);
+
+/*
+ * Options of the _ex attention entry points.  A zeroed struct, or NULL, gives
+ * exactly pkvq_paged_attn_decode / pkvq_paged_attn_prefill.
+ */
+typedef struct {
+    /* > 0: a query at position p sees only keys max(0, p - w + 1) .. p, and
+     * the kernels read no block below the window.  0: keys 0 .. p.  Source:
+     * "1Cat-LLM" README, "DFlash2 Long-Context Decay" (draft attention over
+     * a sliding window of recent keys, the paged loop starting at the
+     * window's first tile). */
+    int32_t sliding_window;
+    /* Decode only (NULL for prefill).  Nullable device int32 [batch][q_len]:
+     * the position of every query among this call's keys, so that key j of
+     * sequence b is visible to query t iff j <= query_pos[b][t] (and
+     * j < context_lens[b]).  NULL means context_lens[b] - q_len + t.  For a
+     * rank holding part of every sequence's keys (sequence-sharded decode,
+     * "ReVolta" PyPI page, "Hardware": TP4 + DCP2): its keys in order, and
+     * for each query the index of the last of them at or before the query's
+     * global position (-1 if none). */
+    const int32_t *query_pos;
+} pkvq_attn_opts;
+
+/*
+ * pkvq_paged_attn_decode with options (sliding window, explicit query
+ * positions).  Same arguments, results and errors otherwise; the workspace
+ * is sized by pkvq_decode_workspace_bytes as before.  sliding_window < 0
+ * returns PKVQ_ERR_INVALID_ARG.
+ */
+PKVQ_API pkvq_status pkvq_paged_attn_decode_ex(const pkvq_cache *cache, const void *q, void *out,
+                                   float *lse_out, const int32_t *block_table,
+                                   int32_t max_blocks_per_seq, const int32_t *context_lens,
+                                   int32_t batch, int32_t q_len, int32_t num_q_heads,
+                                   int32_t max_context_len, float softmax_scale,
+                                   const pkvq_attn_opts *opts, void *workspace,
+                                   size_t workspace_bytes, void *stream);
+
+/*
+ * pkvq_paged_attn_prefill with options (sliding window; query_pos must be
+ * NULL, else PKVQ_ERR_UNSUPPORTED).
+ */
+PKVQ_API pkvq_status pkvq_paged_attn_prefill_ex(const pkvq_cache *cache, const void *q,
+                                    void *out, float *lse_out, const int32_t *cu_seqlens_q,
+                                    const int32_t *block_table, int32_t max_blocks_per_seq,
+                                    const int32_t *context_lens, int32_t batch,
+                                    int32_t max_q_len, int32_t num_q_heads,
+                                    float softmax_scale, const pkvq_attn_opts *opts,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Combines attention results of the same queries computed over disjoint key
+ * sets, e.g. by ranks that each hold part of every sequence's keys, after an
+ * all-gather of their results.  Source: "ReVolta" PyPI page, "Hardware"
+ * (TP4 + DCP2); "1Cat-LLM" README, "Layer 2" (FP32 merge of partial softmax
+ * states).  With lse_r the natural-log sum-exp of part r's scores:
+ *   lse = ln sum_r e^lse_r,  out = sum_r e^(lse_r - lse) out_r  (FP32),
+ * parts with lse_r = -inf (no key) weigh nothing; a row no part saw gets zeros
+ * and lse -inf.
+ *   parts_out  fp16 [num_parts][n_rows][head_dim], each part's normalised output
+ *   parts_lse  fp32 [num_parts][n_rows]
+ *   out        fp16 [n_rows][head_dim];  lse_out nullable fp32 [n_rows]
+ * head_dim must be 128; num_parts 1..64; n_rows == 0 is a no-op.
+ */
+PKVQ_API pkvq_status pkvq_merge_attn_states(const void *parts_out, const float *parts_lse,
+                                   int32_t num_parts, int64_t n_rows, int32_t head_dim,
+                                   void *out, float *lse_out, void *stream);
+
+/*
+ * Copies whole cache blocks between two caches of the same format and block
+ * geometry (dtype, block_size, num_kv_heads, head_dim; the block counts may
+ * differ), e.g. between the GPU pool and a host tier in pinned host memory the
+ * device can address (cudaHostAlloc with mapping, or cudaHostRegister; with
+ * unified addressing the host pointer serves as is).  Source: "ReVolta" PyPI
+ * page, "KV offload modes" (cached pages kept in CPU memory and brought
+ * back).  For i < n, block pairs[2i] of src becomes block pairs[2i + 1] of
+ * dst: its K and V elements and, for INT8, its per-token scales.  The
+ * per-head FP8 scales belong to the cache, not to a block, and are not
+ * copied.  pairs: int32 [n][2], device-addressable.  Destination blocks must
+ * be distinct and none may be a source block of the same call; ids outside
+ * either pool are undefined behaviour (skipped and recorded in a
+ * PKVQ_BOUNDS_CHECK build).  n == 0 is a no-op.
+ */
+PKVQ_API pkvq_status pkvq_kv_copy_blocks(const pkvq_cache *dst, const pkvq_cache *src,
+                                const int32_t *pairs, int32_t n, void *stream);
 
 /* Static description of a status code (never NULL). */
 PKVQ_API const char *pkvq_status_string(pkvq_status status);

@@ -8,11 +8,15 @@ kernels; there is no CPU or PyTorch fallback, and loading fails loudly when
 the library has not been built.
 
 Entry points (same names as the C ABI, without the ``pkvq_`` prefix):
-  kv_write_quant, decode_workspace_bytes, paged_attn_decode,
-  paged_attn_prefill, device_status, status_string, version.
+  kv_write_quant, decode_workspace_bytes, paged_attn_decode (with the _ex
+  options as keyword arguments: sliding_window, query_pos),
+  paged_attn_prefill (sliding_window), merge_attn_states, kv_copy_blocks,
+  device_status, status_string, version.  ``dcp`` adds the all-gather step
+  of sequence-sharded decode (torch.distributed plumbing).
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from dataclasses import dataclass
@@ -26,18 +30,30 @@ LIB_CHECKED_PATH = os.path.join(_HERE, "libpkvq_checked.so")
 
 KV_FP8_E4M3 = 0
 KV_INT8 = 1
+KV_FP8_E5M2 = 2
+KV_FP16 = 3
+_FP8_FORMATS = (KV_FP8_E4M3, KV_FP8_E5M2)
 
 EXPORTED = (
     "pkvq_kv_write_quant",
     "pkvq_decode_workspace_bytes",
     "pkvq_paged_attn_decode",
+    "pkvq_paged_attn_decode_ex",
     "pkvq_paged_attn_decode_noalloc",
     "pkvq_paged_attn_prefill",
+    "pkvq_paged_attn_prefill_ex",
+    "pkvq_merge_attn_states",
+    "pkvq_kv_copy_blocks",
     "pkvq_status_string",
     "pkvq_device_status",
     "pkvq_version",
     "pkvq_last_error",
 )
+
+
+def elem_bytes(dtype: int) -> int:
+    """Bytes per stored cache element of a format (2 for FP16, else 1)."""
+    return 2 if dtype == KV_FP16 else 1
 
 
 class PkvqError(RuntimeError):
@@ -62,6 +78,14 @@ class CacheStruct(ctypes.Structure):
         ("v_scale", ctypes.c_void_p),
         ("k_scale_tok", ctypes.c_void_p),
         ("v_scale_tok", ctypes.c_void_p),
+        ("scale_per_layer", ctypes.c_int32),
+    ]
+
+
+class AttnOpts(ctypes.Structure):
+    _fields_ = [
+        ("sliding_window", ctypes.c_int32),
+        ("query_pos", ctypes.c_void_p),
     ]
 
 
@@ -89,9 +113,19 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pkvq_paged_attn_decode_noalloc.restype = I32
     lib.pkvq_paged_attn_decode_noalloc.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, I32,
                                                    ctypes.c_float, P]
+    lib.pkvq_paged_attn_decode_ex.restype = I32
+    lib.pkvq_paged_attn_decode_ex.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, I32,
+                                              ctypes.c_float, P, P, SZ, P]
     lib.pkvq_paged_attn_prefill.restype = I32
     lib.pkvq_paged_attn_prefill.argtypes = [P, P, P, P, P, P, I32, P, I32, I32, I32,
                                             ctypes.c_float, P, SZ, P]
+    lib.pkvq_paged_attn_prefill_ex.restype = I32
+    lib.pkvq_paged_attn_prefill_ex.argtypes = [P, P, P, P, P, P, I32, P, I32, I32, I32,
+                                               ctypes.c_float, P, P, SZ, P]
+    lib.pkvq_merge_attn_states.restype = I32
+    lib.pkvq_merge_attn_states.argtypes = [P, P, I32, ctypes.c_int64, I32, P, P, P]
+    lib.pkvq_kv_copy_blocks.restype = I32
+    lib.pkvq_kv_copy_blocks.argtypes = [P, P, P, I32, P]
     lib.pkvq_status_string.restype = ctypes.c_char_p
     lib.pkvq_status_string.argtypes = [I32]
     lib.pkvq_device_status.restype = I32
@@ -104,8 +138,23 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     return lib
 
 
+_current = None
+
+
 def _lib():
-    return load_library()
+    return _current if _current is not None else load_library()
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Routes every call of this module to another build of the library
+    (e.g. libpkvq_checked.so, built with PKVQ_BOUNDS_CHECK) inside the block."""
+    global _current
+    prev, _current = _current, load_library(path)
+    try:
+        yield _current
+    finally:
+        _current = prev
 
 
 def status_string(status: int) -> str:
@@ -131,11 +180,13 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _need(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None):
+def _need(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None,
+          host_ok: bool = False):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
+    if not (t.is_cuda or (host_ok and (t.is_pinned() or t.dim() == 1))):
+        raise ValueError(f"{name} must be a CUDA tensor" +
+                         (" or pinned host memory" if host_ok else ""))
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
@@ -146,8 +197,9 @@ def _need(t: torch.Tensor, dtype, name: str, ndim: Optional[int] = None):
 
 @dataclass
 class PagedKVCache:
-    """Caller-owned paged cache: codes [num_blocks][Hkv][block_size][D] uint8
-    (E4M3 bits or int8 two's complement), per-KV-head fp32 scales for FP8,
+    """Caller-owned paged cache: elements [num_blocks][Hkv][block_size][D x
+    elem_bytes] uint8 (E4M3 / E5M2 bits, int8 two's complement, or fp16 bits),
+    fp32 scales for the FP8 formats ([Hkv], or [1] with scale_per_layer),
     per-(block, head, token) fp16 scales for INT8."""
     dtype: int
     k_cache: torch.Tensor
@@ -156,19 +208,31 @@ class PagedKVCache:
     v_scale: Optional[torch.Tensor] = None
     k_scale_tok: Optional[torch.Tensor] = None
     v_scale_tok: Optional[torch.Tensor] = None
+    scale_per_layer: bool = False
 
     @staticmethod
     def allocate(dtype: int, num_blocks: int, block_size: int, num_kv_heads: int,
-                 head_dim: int = 128, device="cuda", k_scale=None, v_scale=None):
-        shape = (num_blocks, num_kv_heads, block_size, head_dim)
-        kc = torch.zeros(shape, dtype=torch.uint8, device=device)
-        vc = torch.zeros(shape, dtype=torch.uint8, device=device)
-        if dtype == KV_FP8_E4M3:
-            ks = torch.as_tensor(k_scale, dtype=torch.float32).to(device).contiguous()
-            vs = torch.as_tensor(v_scale, dtype=torch.float32).to(device).contiguous()
-            return PagedKVCache(dtype, kc, vc, k_scale=ks, v_scale=vs)
-        kst = torch.zeros(shape[:3], dtype=torch.float16, device=device)
-        vst = torch.zeros(shape[:3], dtype=torch.float16, device=device)
+                 head_dim: int = 128, device="cuda", k_scale=None, v_scale=None,
+                 scale_per_layer: bool = False, pin_host: bool = False):
+        """Zeroed cache on `device`; with device="cpu" and pin_host=True, in
+        pinned host memory the GPU can address (a host tier for kv_copy_blocks)."""
+        shape = (num_blocks, num_kv_heads, block_size, head_dim * elem_bytes(dtype))
+
+        def zeros(shp, dt):
+            t = torch.zeros(shp, dtype=dt, device=device)
+            return t.pin_memory() if pin_host else t
+        kc, vc = zeros(shape, torch.uint8), zeros(shape, torch.uint8)
+        if dtype in _FP8_FORMATS:
+            n = 1 if scale_per_layer else num_kv_heads
+            ks = torch.as_tensor(k_scale, dtype=torch.float32).reshape(-1)[:n].to(device)
+            vs = torch.as_tensor(v_scale, dtype=torch.float32).reshape(-1)[:n].to(device)
+            if ks.numel() != n or vs.numel() != n:
+                raise ValueError(f"need {n} K and V scales")
+            return PagedKVCache(dtype, kc, vc, k_scale=ks.contiguous(), v_scale=vs.contiguous(),
+                                scale_per_layer=scale_per_layer)
+        if dtype == KV_FP16:
+            return PagedKVCache(dtype, kc, vc)
+        kst, vst = zeros(shape[:3], torch.float16), zeros(shape[:3], torch.float16)
         return PagedKVCache(dtype, kc, vc, k_scale_tok=kst, v_scale_tok=vst)
 
     @property
@@ -185,24 +249,26 @@ class PagedKVCache:
 
     @property
     def head_dim(self):
-        return self.k_cache.shape[3]
+        return self.k_cache.shape[3] // elem_bytes(self.dtype)
 
-    def struct(self) -> CacheStruct:
+    def struct(self, device_ok: bool = False) -> CacheStruct:
         for name in ("k_cache", "v_cache"):
-            _need(getattr(self, name), torch.uint8, name, 4)
-        if self.dtype == KV_FP8_E4M3:
-            _need(self.k_scale, torch.float32, "k_scale", 1)
-            _need(self.v_scale, torch.float32, "v_scale", 1)
-        else:
-            _need(self.k_scale_tok, torch.float16, "k_scale_tok", 3)
-            _need(self.v_scale_tok, torch.float16, "v_scale_tok", 3)
-        nb, hkv, bs, d = self.k_cache.shape
-        return CacheStruct(self.dtype, nb, bs, hkv, d,
+            _need(getattr(self, name), torch.uint8, name, 4, host_ok=device_ok)
+        if self.dtype in _FP8_FORMATS:
+            # (a block copy reads no scale: a host tier may keep its own copy)
+            _need(self.k_scale, torch.float32, "k_scale", 1, host_ok=device_ok)
+            _need(self.v_scale, torch.float32, "v_scale", 1, host_ok=device_ok)
+        elif self.dtype == KV_INT8:
+            _need(self.k_scale_tok, torch.float16, "k_scale_tok", 3, host_ok=device_ok)
+            _need(self.v_scale_tok, torch.float16, "v_scale_tok", 3, host_ok=device_ok)
+        nb, hkv, bs, rb = self.k_cache.shape
+        return CacheStruct(self.dtype, nb, bs, hkv, rb // elem_bytes(self.dtype),
                            self.k_cache.data_ptr(), self.v_cache.data_ptr(),
                            self.k_scale.data_ptr() if self.k_scale is not None else None,
                            self.v_scale.data_ptr() if self.v_scale is not None else None,
                            self.k_scale_tok.data_ptr() if self.k_scale_tok is not None else None,
-                           self.v_scale_tok.data_ptr() if self.v_scale_tok is not None else None)
+                           self.v_scale_tok.data_ptr() if self.v_scale_tok is not None else None,
+                           1 if self.scale_per_layer else 0)
 
 
 def kv_write_quant(cache: PagedKVCache, k: torch.Tensor, v: torch.Tensor,
@@ -224,11 +290,21 @@ def decode_workspace_bytes(cache: PagedKVCache, batch: int, q_len: int, num_q_he
                                                   ctypes.byref(cs)))
 
 
+def _opts(sliding_window: int, query_pos: Optional[torch.Tensor]):
+    if not sliding_window and query_pos is None:
+        return None
+    return AttnOpts(int(sliding_window), None if query_pos is None else query_pos.data_ptr())
+
+
 def paged_attn_decode(cache: PagedKVCache, q: torch.Tensor, block_table: torch.Tensor,
                       context_lens: torch.Tensor, max_context_len: int, softmax_scale: float,
                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                      workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """q fp16 [B][q_len][Hq][D] -> out fp16 [B][q_len][Hq][D] (lse fp32 [B][q_len][Hq])."""
+                      workspace: Optional[torch.Tensor] = None, stream=None,
+                      sliding_window: int = 0,
+                      query_pos: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """q fp16 [B][q_len][Hq][D] -> out fp16 [B][q_len][Hq][D] (lse fp32 [B][q_len][Hq]).
+    sliding_window > 0 limits every query to its last `sliding_window` keys;
+    query_pos (int32 [B][q_len]) gives each query's position among the keys."""
     _need(q, torch.float16, "q", 4)
     _need(block_table, torch.int32, "block_table", 2)
     _need(context_lens, torch.int32, "context_lens", 1)
@@ -238,22 +314,29 @@ def paged_attn_decode(cache: PagedKVCache, q: torch.Tensor, block_table: torch.T
     _need(out, torch.float16, "out", 4)
     if lse is not None:
         _need(lse, torch.float32, "lse", 3)
+    if query_pos is not None:
+        _need(query_pos, torch.int32, "query_pos", 2)
+        if tuple(query_pos.shape) != (B, q_len):
+            raise ValueError("query_pos must be [batch][q_len]")
     need = decode_workspace_bytes(cache, B, q_len, Hq, max_context_len) if B else 0
-    if workspace is None and need:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is None and need:   # zero-filled before its first use
+        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     cs = cache.struct()
-    _check(_lib().pkvq_paged_attn_decode(
+    opts = _opts(sliding_window, query_pos)
+    _check(_lib().pkvq_paged_attn_decode_ex(
         ctypes.byref(cs), _ptr(q), _ptr(out), _ptr(lse), _ptr(block_table),
         int(block_table.shape[1]), _ptr(context_lens), B, q_len, Hq, int(max_context_len),
-        float(softmax_scale), _ptr(workspace), wbytes, _stream(stream)), "paged_attn_decode")
+        float(softmax_scale), None if opts is None else ctypes.byref(opts), _ptr(workspace),
+        wbytes, _stream(stream)), "paged_attn_decode")
     return out
 
 
 def paged_attn_prefill(cache: PagedKVCache, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
                        block_table: torch.Tensor, context_lens: torch.Tensor, max_q_len: int,
                        softmax_scale: float, out: Optional[torch.Tensor] = None,
-                       lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                       lse: Optional[torch.Tensor] = None, stream=None,
+                       sliding_window: int = 0) -> torch.Tensor:
     """q fp16 [total_q][Hq][D] (packed varlen) -> out fp16 [total_q][Hq][D]."""
     _need(q, torch.float16, "q", 3)
     _need(cu_seqlens_q, torch.int32, "cu_seqlens_q", 1)
@@ -267,11 +350,45 @@ def paged_attn_prefill(cache: PagedKVCache, q: torch.Tensor, cu_seqlens_q: torch
         _need(lse, torch.float32, "lse", 2)
     B = int(context_lens.shape[0])
     cs = cache.struct()
-    _check(_lib().pkvq_paged_attn_prefill(
+    opts = _opts(sliding_window, None)
+    _check(_lib().pkvq_paged_attn_prefill_ex(
         ctypes.byref(cs), _ptr(q), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q), _ptr(block_table),
         int(block_table.shape[1]), _ptr(context_lens), B, int(max_q_len), Hq,
-        float(softmax_scale), None, 0, _stream(stream)), "paged_attn_prefill")
+        float(softmax_scale), None if opts is None else ctypes.byref(opts), None, 0,
+        _stream(stream)), "paged_attn_prefill")
     return out
+
+
+def merge_attn_states(parts_out: torch.Tensor, parts_lse: torch.Tensor,
+                      out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                      stream=None):
+    """parts_out fp16 [R][..., D], parts_lse fp32 [R][...] (results of the same
+    queries over disjoint key sets) -> (out fp16 [..., D], lse fp32 [...])."""
+    _need(parts_out, torch.float16, "parts_out")
+    _need(parts_lse, torch.float32, "parts_lse")
+    R, D = int(parts_out.shape[0]), int(parts_out.shape[-1])
+    if tuple(parts_lse.shape) != tuple(parts_out.shape[:-1]):
+        raise ValueError("parts_lse must match parts_out without its last dimension")
+    n = parts_lse.numel() // max(R, 1)
+    if out is None:
+        out = torch.empty(parts_out.shape[1:], dtype=torch.float16, device=parts_out.device)
+    if lse is None:
+        lse = torch.empty(parts_lse.shape[1:], dtype=torch.float32, device=parts_out.device)
+    _need(out, torch.float16, "out")
+    _need(lse, torch.float32, "lse")
+    _check(_lib().pkvq_merge_attn_states(_ptr(parts_out), _ptr(parts_lse), R, n, D, _ptr(out),
+                                         _ptr(lse), _stream(stream)), "merge_attn_states")
+    return out, lse
+
+
+def kv_copy_blocks(dst: PagedKVCache, src: PagedKVCache, pairs: torch.Tensor,
+                   stream=None) -> None:
+    """Block pairs[i][0] of src -> block pairs[i][1] of dst (either cache on the
+    GPU or in pinned host memory; pairs int32 [n][2] on the GPU)."""
+    _need(pairs, torch.int32, "pairs", 2)
+    sd, ss = dst.struct(device_ok=True), src.struct(device_ok=True)
+    _check(_lib().pkvq_kv_copy_blocks(ctypes.byref(sd), ctypes.byref(ss), _ptr(pairs),
+                                      int(pairs.shape[0]), _stream(stream)), "kv_copy_blocks")
 
 
 def device_status(clear: bool = True) -> int:

@@ -61,7 +61,8 @@ pkvq_status check_cache(const pkvq_cache *c)
 {
     if (!c || !c->k_cache || !c->v_cache)
         return PKVQ_ERR_INVALID_ARG;
-    if (c->dtype != PKVQ_KV_FP8_E4M3 && c->dtype != PKVQ_KV_INT8)
+    if (c->dtype != PKVQ_KV_FP8_E4M3 && c->dtype != PKVQ_KV_INT8 &&
+        c->dtype != PKVQ_KV_FP8_E5M2 && c->dtype != PKVQ_KV_FP16)
         return PKVQ_ERR_UNSUPPORTED;
     if (c->head_dim != kHeadDim)
         return PKVQ_ERR_UNSUPPORTED;
@@ -72,10 +73,10 @@ pkvq_status check_cache(const pkvq_cache *c)
     // tensor-map row coordinates are int32
     if ((long long)c->num_blocks * c->num_kv_heads * c->block_size >= (1LL << 31))
         return PKVQ_ERR_UNSUPPORTED;
-    if (c->dtype == PKVQ_KV_FP8_E4M3) {
+    if (kv_has_head_scale(c->dtype)) {
         if (!c->k_scale || !c->v_scale)
             return PKVQ_ERR_INVALID_ARG;
-    } else {
+    } else if (c->dtype == PKVQ_KV_INT8) {
         if (!c->k_scale_tok || !c->v_scale_tok)
             return PKVQ_ERR_INVALID_ARG;
         if (!aligned16(c->k_scale_tok) || !aligned16(c->v_scale_tok))
@@ -89,10 +90,16 @@ pkvq_status check_cache(const pkvq_cache *c)
 pkvq_status cache_maps(const pkvq_cache *c, CUtensorMap *km, CUtensorMap *vm)
 {
     const uint64_t rows = (uint64_t)c->num_blocks * c->num_kv_heads * c->block_size;
-    if (!make_cache_tensor_map(km, c->k_cache, rows, c->block_size) ||
-        !make_cache_tensor_map(vm, c->v_cache, rows, c->block_size))
+    const int row_bytes = kHeadDim * kv_elem_bytes(c->dtype);
+    if (!make_cache_tensor_map(km, c->k_cache, rows, c->block_size, row_bytes) ||
+        !make_cache_tensor_map(vm, c->v_cache, rows, c->block_size, row_bytes))
         return PKVQ_ERR_CUDA;
     return PKVQ_OK;
+}
+
+int scale_stride(const pkvq_cache *c)
+{
+    return c->scale_per_layer ? 0 : 1;
 }
 
 thread_local char t_last_error[256] = "";
@@ -110,13 +117,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 }  // namespace
 
-bool make_cache_tensor_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows)
+bool make_cache_tensor_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows,
+                           int row_bytes)
 {
     auto fn = encode_fn();
     if (!fn)
         return false;
-    cuuint64_t dims[2] = {128, rows};
-    cuuint64_t strides[1] = {128};
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
     cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
@@ -203,6 +211,7 @@ pkvq_status pkvq_kv_write_quant(const pkvq_cache *cache, const void *k, const vo
     p.v_cache = static_cast<uint8_t *>(cache->v_cache);
     p.k_scale = cache->k_scale;
     p.v_scale = cache->v_scale;
+    p.scale_stride = scale_stride(cache);
     p.k_scale_tok = static_cast<uint16_t *>(cache->k_scale_tok);
     p.v_scale_tok = static_cast<uint16_t *>(cache->v_scale_tok);
     p.k = static_cast<const __half *>(k);
@@ -238,6 +247,21 @@ pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void *q, void 
                                    int32_t max_context_len, float softmax_scale,
                                    void *workspace, size_t workspace_bytes, void *stream)
 {
+    return pkvq_paged_attn_decode_ex(cache, q, out, lse_out, block_table, max_blocks_per_seq,
+                                     context_lens, batch, q_len, num_q_heads, max_context_len,
+                                     softmax_scale, nullptr, workspace, workspace_bytes, stream);
+}
+
+pkvq_status pkvq_paged_attn_decode_ex(const pkvq_cache *cache, const void *q, void *out,
+                                      float *lse_out, const int32_t *block_table,
+                                      int32_t max_blocks_per_seq, const int32_t *context_lens,
+                                      int32_t batch, int32_t q_len, int32_t num_q_heads,
+                                      int32_t max_context_len, float softmax_scale,
+                                      const pkvq_attn_opts *opts, void *workspace,
+                                      size_t workspace_bytes, void *stream)
+{
+    if (opts && opts->sliding_window < 0)
+        return PKVQ_ERR_INVALID_ARG;
     pkvq_status st = check_cache(cache);
     if (st != PKVQ_OK)
         return st;
@@ -274,10 +298,14 @@ pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void *q, void 
     if (st != PKVQ_OK)
         return st;
     DecodeParams p{};
-    p.k_scale = cache->k_scale;
-    p.v_scale = cache->dtype == PKVQ_KV_FP8_E4M3 ? cache->v_scale : nullptr;
+    const bool head_scale = kv_has_head_scale(cache->dtype);
+    p.k_scale = head_scale ? cache->k_scale : nullptr;
+    p.v_scale = head_scale ? cache->v_scale : nullptr;
+    p.scale_stride = scale_stride(cache);
     p.k_scale_tok = static_cast<const uint16_t *>(cache->k_scale_tok);
     p.v_scale_tok = static_cast<const uint16_t *>(cache->v_scale_tok);
+    p.window = opts ? opts->sliding_window : 0;
+    p.query_pos = opts ? opts->query_pos : nullptr;
     p.q = static_cast<const __half *>(q);
     p.out = static_cast<__half *>(out);
     p.lse = lse_out;
@@ -300,11 +328,13 @@ pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void *q, void 
     p.split_min_blocks = plan.split_min_blocks;
     p.split_gran = plan.split_gran;
     p.scale_log2 = softmax_scale * kLog2e;
-    float *ws = static_cast<float *>(workspace);
+    // workspace: [arrival counters][partial O][partial (m, l)]
+    float *ws = reinterpret_cast<float *>(static_cast<char *>(workspace) + plan.counters_bytes);
     const size_t n_rows_ws = (size_t)cache->num_kv_heads * plan.row_groups * plan.num_splits *
                              plan.rows_per_cta;
     p.ws_o = plan.workspace_bytes ? ws : nullptr;
     p.ws_ml = plan.workspace_bytes ? ws + n_rows_ws * kHeadDim : nullptr;
+    p.ws_cnt = plan.fused_merge ? static_cast<int *>(workspace) : nullptr;
     p.status = status_ptr();
     if (!p.status)
         return PKVQ_ERR_CUDA;
@@ -319,8 +349,26 @@ pkvq_status pkvq_paged_attn_prefill(const pkvq_cache *cache, const void *q, void
                                     float softmax_scale, void *workspace,
                                     size_t workspace_bytes, void *stream)
 {
+    return pkvq_paged_attn_prefill_ex(cache, q, out, lse_out, cu_seqlens_q, block_table,
+                                      max_blocks_per_seq, context_lens, batch, max_q_len,
+                                      num_q_heads, softmax_scale, nullptr, workspace,
+                                      workspace_bytes, stream);
+}
+
+pkvq_status pkvq_paged_attn_prefill_ex(const pkvq_cache *cache, const void *q, void *out,
+                                       float *lse_out, const int32_t *cu_seqlens_q,
+                                       const int32_t *block_table, int32_t max_blocks_per_seq,
+                                       const int32_t *context_lens, int32_t batch,
+                                       int32_t max_q_len, int32_t num_q_heads,
+                                       float softmax_scale, const pkvq_attn_opts *opts,
+                                       void *workspace, size_t workspace_bytes, void *stream)
+{
     (void)workspace;
     (void)workspace_bytes;
+    if (opts && opts->sliding_window < 0)
+        return PKVQ_ERR_INVALID_ARG;
+    if (opts && opts->query_pos)
+        return PKVQ_ERR_UNSUPPORTED;
     pkvq_status st = check_cache(cache);
     if (st != PKVQ_OK)
         return st;
@@ -344,8 +392,11 @@ pkvq_status pkvq_paged_attn_prefill(const pkvq_cache *cache, const void *q, void
     if (st != PKVQ_OK)
         return st;
     PrefillParams p{};
-    p.k_scale = cache->k_scale;
-    p.v_scale = cache->v_scale;
+    const bool head_scale = kv_has_head_scale(cache->dtype);
+    p.k_scale = head_scale ? cache->k_scale : nullptr;
+    p.v_scale = head_scale ? cache->v_scale : nullptr;
+    p.scale_stride = scale_stride(cache);
+    p.window = opts ? opts->sliding_window : 0;
     p.k_scale_tok = static_cast<const uint16_t *>(cache->k_scale_tok);
     p.v_scale_tok = static_cast<const uint16_t *>(cache->v_scale_tok);
     p.q = static_cast<const __half *>(q);
@@ -369,6 +420,71 @@ pkvq_status pkvq_paged_attn_prefill(const pkvq_cache *cache, const void *q, void
     if (!p.status)
         return PKVQ_ERR_CUDA;
     return from_cuda(launch_prefill_tc(p, cache->dtype, km, vm, static_cast<cudaStream_t>(stream)));
+}
+
+pkvq_status pkvq_merge_attn_states(const void *parts_out, const float *parts_lse,
+                                   int32_t num_parts, int64_t n_rows, int32_t head_dim,
+                                   void *out, float *lse_out, void *stream)
+{
+    if (head_dim != kHeadDim)
+        return PKVQ_ERR_UNSUPPORTED;
+    if (num_parts < 1 || num_parts > 64 || n_rows < 0)
+        return PKVQ_ERR_INVALID_ARG;
+    if (n_rows == 0)
+        return PKVQ_OK;
+    if (!parts_out || !parts_lse || !out)
+        return PKVQ_ERR_INVALID_ARG;
+    if (!aligned16(parts_out) || !aligned16(out))
+        return PKVQ_ERR_MISALIGNED;
+    MergeParams p{};
+    p.parts_out = static_cast<const __half *>(parts_out);
+    p.parts_lse = parts_lse;
+    p.out = static_cast<__half *>(out);
+    p.lse = lse_out;
+    p.parts = num_parts;
+    p.rows = n_rows;
+    return from_cuda(launch_merge_states(p, static_cast<cudaStream_t>(stream)));
+}
+
+pkvq_status pkvq_kv_copy_blocks(const pkvq_cache *dst, const pkvq_cache *src,
+                                const int32_t *pairs, int32_t n, void *stream)
+{
+    pkvq_status st = check_cache(dst);
+    if (st != PKVQ_OK)
+        return st;
+    st = check_cache(src);
+    if (st != PKVQ_OK)
+        return st;
+    if (dst->dtype != src->dtype || dst->block_size != src->block_size ||
+        dst->num_kv_heads != src->num_kv_heads || dst->head_dim != src->head_dim)
+        return PKVQ_ERR_INVALID_ARG;
+    if (n < 0)
+        return PKVQ_ERR_INVALID_ARG;
+    if (n == 0)
+        return PKVQ_OK;
+    if (!pairs)
+        return PKVQ_ERR_INVALID_ARG;
+    CopyParams p{};
+    p.src_k = static_cast<const uint8_t *>(src->k_cache);
+    p.src_v = static_cast<const uint8_t *>(src->v_cache);
+    p.dst_k = static_cast<uint8_t *>(dst->k_cache);
+    p.dst_v = static_cast<uint8_t *>(dst->v_cache);
+    const bool int8 = src->dtype == PKVQ_KV_INT8;
+    p.src_ks = int8 ? static_cast<const uint16_t *>(src->k_scale_tok) : nullptr;
+    p.src_vs = int8 ? static_cast<const uint16_t *>(src->v_scale_tok) : nullptr;
+    p.dst_ks = int8 ? static_cast<uint16_t *>(dst->k_scale_tok) : nullptr;
+    p.dst_vs = int8 ? static_cast<uint16_t *>(dst->v_scale_tok) : nullptr;
+    p.pairs = pairs;
+    p.n = n;
+    p.block_bytes = (long long)src->num_kv_heads * src->block_size * kHeadDim *
+                    kv_elem_bytes(src->dtype);
+    p.block_scales = int8 ? src->num_kv_heads * src->block_size : 0;
+    p.src_blocks = src->num_blocks;
+    p.dst_blocks = dst->num_blocks;
+    p.status = status_ptr();
+    if (!p.status)
+        return PKVQ_ERR_CUDA;
+    return from_cuda(launch_copy_blocks(p, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -219,6 +219,18 @@ __device__ __forceinline__ void e4m3x4_to_half2x2(uint32_t x, uint32_t &lo, uint
         : "r"(x));
 }
 
+// Four E5M2 codes (bytes b0..b3 of x) -> half2 (b0, b1) and half2 (b2, b3).
+// Exact: an E5M2 code is the high byte of the fp16 with the same value.
+__device__ __forceinline__ void e5m2x4_to_half2x2(uint32_t x, uint32_t &lo, uint32_t &hi)
+{
+    asm("{\n\t.reg .b16 a, b;\n\t"
+        "mov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e5m2x2 %0, a;\n\t"
+        "cvt.rn.f16x2.e5m2x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(x));
+}
+
 // Four int8 codes (bytes b0..b3 of x) -> half2 (b0, b1) and half2 (b2, b3),
 // exact (see s8x2_to_half2).
 __device__ __forceinline__ void s8x4_to_half2x2(uint32_t x, uint32_t &lo, uint32_t &hi)
@@ -229,6 +241,23 @@ __device__ __forceinline__ void s8x4_to_half2x2(uint32_t x, uint32_t &lo, uint32
     const __half2 k = __half2half2(__ushort_as_half(0x6480));   // 1152
     __half2 lh = __hsub2(*reinterpret_cast<__half2 *>(&l), k);
     __half2 hh = __hsub2(*reinterpret_cast<__half2 *>(&h), k);
+    lo = *reinterpret_cast<uint32_t *>(&lh);
+    hi = *reinterpret_cast<uint32_t *>(&hh);
+}
+
+// Four int8 codes -> half2 (b0, b1) and (b2, b3) of code * 2^e, with
+// p2 = 2^e and nb2 = -1152 * 2^e (both exact in fp16): the magic-number form
+// (1152 + code) times 2^e minus 1152 * 2^e in one fused multiply-add, whose
+// exact result code * 2^e is representable, so it is exact whenever
+// |code * 2^e| stays below 65504.
+__device__ __forceinline__ void s8x4_to_half2x2_scaled(uint32_t x, __half2 p2, __half2 nb2,
+                                                       uint32_t &lo, uint32_t &hi)
+{
+    const uint32_t biased = x ^ 0x80808080u;
+    uint32_t l = __byte_perm(biased, 0x64646464u, 0x5140);
+    uint32_t h = __byte_perm(biased, 0x64646464u, 0x7362);
+    __half2 lh = __hfma2(*reinterpret_cast<__half2 *>(&l), p2, nb2);
+    __half2 hh = __hfma2(*reinterpret_cast<__half2 *>(&h), p2, nb2);
     lo = *reinterpret_cast<uint32_t *>(&lh);
     hi = *reinterpret_cast<uint32_t *>(&hh);
 }

@@ -28,11 +28,19 @@
 // reads 32 contiguous code bytes per key.  P^T reaches the B-operand layout
 // through movmatrix.trans, without shared memory.
 //
-// Scales.  FP8: the per-head K scale folds into the score multiplier and the
-// per-head V scale into the final normalisation.  INT8: the per-token K scale
-// multiplies score columns in fp32; the per-token V scale multiplies the
-// dequantised V in fp16 before the PV product (P itself stays unscaled, so
-// small probabilities never meet small scales in fp16).
+// Scales.  FP8 (E4M3, E5M2): the per-head (or per-layer) K scale folds into
+// the score multiplier and the V scale into the final normalisation.  INT8:
+// the per-token K scale multiplies score columns in fp32; the per-token V
+// scale multiplies the dequantised V in fp16 before the PV product (P itself
+// stays unscaled, so small probabilities never meet small scales in fp16).
+// FP16 caches hold the values themselves: a row of 128 values is 256 bytes,
+// fetched as two 128-byte-wide boxes (d 0-63, d 64-127) and read straight
+// into the MMA fragments.
+//
+// Visibility.  Key j is visible to a query row at position pos iff j <= pos,
+// j < context length and, with a sliding window w, j > pos - w ("1Cat-LLM"
+// README, "DFlash2 Long-Context Decay").  Positions are context - q_len + t,
+// or given per query (a rank holding part of each sequence's keys).
 #include "common.cuh"
 #include "internal.h"
 #include "split_map.cuh"
@@ -46,21 +54,25 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr float kLn2 = 0.693147180559945309f;
 
-template <int BS>
+template <int KVT, int BS>
 struct DecodeCfg {
-    static constexpr int kStages = BS == 16 ? 4 : (BS == 32 ? 3 : 2);
-    static constexpr int kUnroll = BS == 16 ? 2 : 1;   // cache blocks per loop iteration
-    static constexpr int kTileBytes = BS * 128;
+    static constexpr int kEB = kv_elem_bytes(KVT);
+    // bytes of one (block, head) tile per warp stage; FP16 tiles are twice as
+    // large, so they take fewer stages
+    static constexpr int kTileBytes = BS * 128 * kEB;
     static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kStages =
+        kEB == 1 ? (BS == 16 ? 4 : (BS == 32 ? 3 : 2)) : (BS == 16 ? 3 : (BS == 32 ? 2 : 1));
+    static constexpr int kUnroll = (BS == 16 && kEB == 1) ? 2 : 1;   // blocks per loop iteration
     static constexpr int kScaleHalves = 2 * BS;     // K then V scales of one block
     static constexpr int kMT = BS / 16;             // 16-key m-tiles per block
-    static_assert(kStages >= 2 * kUnroll, "ring must hold two iterations");
+    static_assert(kStages >= kUnroll, "ring must hold one iteration");
 };
 
-template <int BS>
+template <int KVT, int BS>
 constexpr size_t decode_smem_bytes()
 {
-    using C = DecodeCfg<BS>;
+    using C = DecodeCfg<KVT, BS>;
     return 1024 + (size_t)kWarps * C::kStages * C::kStageBytes +
            (size_t)kWarps * C::kStages * C::kScaleHalves * 2 + (size_t)kWarps * C::kStages * 8;
 }
@@ -75,6 +87,8 @@ __device__ __forceinline__ void cvt4(uint32_t x, uint32_t &lo, uint32_t &hi)
 {
     if constexpr (KVT == kKvFp8)
         e4m3x4_to_half2x2(x, lo, hi);
+    else if constexpr (KVT == kKvE5m2)
+        e5m2x4_to_half2x2(x, lo, hi);
     else
         s8x4_to_half2x2(x, lo, hi);
 }
@@ -194,6 +208,174 @@ __device__ __forceinline__ void pv_block(const uint8_t *vt, const uint16_t *st, 
     }
 }
 
+// FP16 cache, S^T = K Q^T for one block.  A key row is two 128-byte halves
+// (d 0-63 at the tile's start, d 64-127 at + BS * 128), each 128-byte
+// swizzled.  Lane (g, t) reads d = 32t .. 32t+31 of keys g and g+8: chunks
+// 4(t&1) .. 4(t&1)+3 of half t>>1; the A fragment of k-step ks is word
+// 2(ks&1) (d 32t+4ks, +1) and word 2(ks&1)+1 (d +2, +3) of chunk ks>>1, the
+// same d order as the 8-bit path, so Q's fragments serve both.
+template <int NT, int MT, int BS>
+__device__ __forceinline__ void qk_block_f16(const uint8_t *kt, int g, int t,
+                                             const uint32_t (&qf)[NT][8][2], float kfac,
+                                             float (&sc)[MT][NT][4])
+{
+    const uint8_t *half = kt + (t >> 1) * BS * 128;
+    const int c0 = 4 * (t & 1);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int r0 = mt * 16 + g;   // rows r0, r0 + 8 share (row & 7) == g
+        uint4 ka[4], kb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            ka[i] = lds128(half + r0 * 128 + (((c0 + i) ^ g) << 4));
+            kb[i] = lds128(half + (r0 + 8) * 128 + (((c0 + i) ^ g) << 4));
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                sc[mt][nt][c] = 0.0f;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint4 &wa = ka[ks >> 1], &wb = kb[ks >> 1];
+            uint32_t a[4];
+            a[0] = (ks & 1) ? wa.z : wa.x;
+            a[2] = (ks & 1) ? wa.w : wa.y;
+            a[1] = (ks & 1) ? wb.z : wb.x;
+            a[3] = (ks & 1) ? wb.w : wb.y;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                mma_f16_16816(sc[mt][nt], a, qf[nt][ks]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                sc[mt][nt][c] *= kfac;
+    }
+}
+
+// FP16 cache, O^T += V^T P^T for one block.  Lane (g, t) reads d = 16g ..
+// 16g+15 (chunks 2(g&3), 2(g&3)+1 of half g>>2) of keys 2t, 2t+1, 2t+8, 2t+9;
+// word w of that range is d-tile w: row g <-> d = 16g+2w, row g+8 <-> +1, the
+// same output order as the 8-bit path.
+template <int NT, int MT, int BS>
+__device__ __forceinline__ void pv_block_f16(const uint8_t *vt, int g, int t, int key0, int ctx,
+                                             const float (&pr)[MT][NT][4],
+                                             float (&o)[NT][8][4])
+{
+    const uint8_t *half = vt + (g >> 2) * BS * 128;
+    const int c0 = 2 * (g & 3);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        uint32_t pb[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            pb[nt][0] = movmatrix_trans(pack_half2(pr[mt][nt][0], pr[mt][nt][1]));
+            pb[nt][1] = movmatrix_trans(pack_half2(pr[mt][nt][2], pr[mt][nt][3]));
+        }
+        const int r0 = mt * 16 + 2 * t;   // key rows r0, r0+1, r0+8, r0+9
+        const int rr[4] = {r0, r0 + 1, r0 + 8, r0 + 9};
+        uint4 v[4][2];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+                v[k][j] = lds128(half + rr[k] * 128 + (((c0 + j) ^ (rr[k] & 7)) << 4));
+        if (key0 + BS > ctx) {
+            // Slots past the context were never written: their values may be
+            // NaN patterns, and 0 * NaN would poison O.
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (key0 + rr[k] >= ctx)
+                    v[k][0] = v[k][1] = make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            const uint32_t x0 = word_of(v[0][w >> 2], w & 3), x1 = word_of(v[1][w >> 2], w & 3);
+            const uint32_t x2 = word_of(v[2][w >> 2], w & 3), x3 = word_of(v[3][w >> 2], w & 3);
+            uint32_t a[4];
+            a[0] = __byte_perm(x0, x1, 0x5410);   // d = 16g+2w of keys r0, r0+1
+            a[1] = __byte_perm(x0, x1, 0x7632);   // d + 1
+            a[2] = __byte_perm(x2, x3, 0x5410);
+            a[3] = __byte_perm(x2, x3, 0x7632);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+                mma_f16_16816(o[nt][w], a, pb[nt]);
+        }
+    }
+}
+
+// Merge of the split partial states of one output row by one warp:
+// M = max_i m_i, L = sum_i l_i 2^(m_i - M), O = sum_i O_i 2^(m_i - M) / L.
+// The splits are taken kMergeChunk at a time: every lane issues the loads of
+// a whole chunk (the (m, l) pairs, the same for all lanes, and its float4 of
+// each O row) before using any, so a chunk costs one memory round trip; the
+// chunks are combined online.  `preloaded`: the caller already loaded the
+// first chunk for slots first .. (ml, v).
+constexpr int kMergeChunk = 16;
+
+struct MergeRow {
+    size_t row0, stride;   // workspace row of the first slot, rows between slots
+    float2 ml[kMergeChunk];
+    float4 v[kMergeChunk];
+
+    __device__ __forceinline__ void load(const DecodeParams &p, int first, int nsplit, int s0,
+                                         int lane)
+    {
+#pragma unroll
+        for (int k = 0; k < kMergeChunk; ++k) {
+            ml[k] = make_float2(-INFINITY, 0.0f);
+            v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (s0 + k < nsplit && first + s0 + k < p.num_splits) {
+                const size_t wrow = row0 + (size_t)(first + s0 + k) * stride;
+                ml[k] = *reinterpret_cast<const float2 *>(p.ws_ml + wrow * 2);
+                v[k] = reinterpret_cast<const float4 *>(p.ws_o + wrow * kHeadDim)[lane];
+            }
+        }
+    }
+
+    // Combines the nsplit partials (the first chunk already loaded) and
+    // writes output row rr of sequence b, KV head h.
+    __device__ __forceinline__ void finish(const DecodeParams &p, int first, int nsplit, int b,
+                                           int h, int rr, int lane)
+    {
+        float M = -INFINITY, L = 0.0f;
+        float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = 0; s0 < nsplit; s0 += kMergeChunk) {
+            if (s0 > 0)
+                load(p, first, nsplit, s0, lane);
+            float cm = M;
+#pragma unroll
+            for (int k = 0; k < kMergeChunk; ++k)
+                cm = fmaxf(cm, ml[k].x);
+            const float mu = cm == -INFINITY ? 0.0f : cm;
+            const float corr = fast_exp2(M - mu);
+            L *= corr;
+            O.x *= corr, O.y *= corr, O.z *= corr, O.w *= corr;
+#pragma unroll
+            for (int k = 0; k < kMergeChunk; ++k) {
+                const float e = fast_exp2(ml[k].x - mu);
+                L += ml[k].y * e;
+                O.x += v[k].x * e, O.y += v[k].y * e, O.z += v[k].z * e, O.w += v[k].w * e;
+            }
+            M = cm;
+        }
+        const float vfac = p.v_scale ? __ldg(p.v_scale + h * p.scale_stride) : 1.0f;
+        const float f = L > 0.0f ? vfac / L : 0.0f;
+        const int tq = rr / p.group, gq = rr % p.group;
+        const size_t orow = ((size_t)b * p.q_len + tq) * p.num_q_heads + h * p.group + gq;
+        const __half2 lo = __floats2half2_rn(O.x * f, O.y * f);
+        const __half2 hi = __floats2half2_rn(O.z * f, O.w * f);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t *>(&lo);
+        pk.y = *reinterpret_cast<const uint32_t *>(&hi);
+        reinterpret_cast<uint2 *>(p.out + orow * kHeadDim)[lane] = pk;
+        if (lane == 0 && p.lse)
+            p.lse[orow] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+};
+
 constexpr int kMinBlocksPerWarp = 3;   // shortest split: 3 cache blocks per warp
 
 template <int KVT, int NT, int BS>
@@ -201,7 +383,7 @@ __global__ void __launch_bounds__(kThreads)
 decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap, const DecodeParams p)
 {
-    using C = DecodeCfg<BS>;
+    using C = DecodeCfg<KVT, BS>;
     constexpr int S = C::kStages;
     constexpr int U = C::kUnroll;
     constexpr int RC = 8 * NT;
@@ -240,7 +422,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     // to finish before reading the workspace.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    if (device_wait_failed(p.status))
+    // (a CTA-wide decision: the kernel ends with CTA barriers)
+    if (__syncthreads_or(device_wait_failed(p.status)))
         return;
     // The block ids of this warp's first 64 iterations and the query rows are
     // loaded for a guess of this slot's (sequence, split): the assignment all
@@ -293,7 +476,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     const SplitInfo si = find_split<BS>(p, slot, -1);
     if (si.b < 0)
         return;   // a slot past the last split: no work
-    const int real_begin = si.split * si.bpc;
+    const int real_begin = si.blk0 + si.split * si.bpc;
     if (si.b != b || real_begin != blk_begin) {
         const bool new_seq = si.b != b;
         b = si.b;
@@ -307,18 +490,31 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     const int nblk = max(0, min(nblk_seq, blk_begin + si.bpc) - blk_begin);
     const int n_it = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
     const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq;
-    int pos[NT][2];
+    // each thread's two rows per n8 tile: last visible key (pos) and first
+    // (lo); padding rows see the whole split
+    int pos[NT][2], lo[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             const int rr = rg * RC + nt * 8 + 2 * t + i;
-            pos[nt][i] = rr < p.rows ? ctx - p.q_len + rr / p.group : ctx - 1;
+            pos[nt][i] = rr < p.rows ? min(ctx - 1, query_position(p, b, ctx, rr / p.group))
+                                     : ctx - 1;
+            lo[nt][i] = p.window > 0 && rr < p.rows ? pos[nt][i] - p.window + 1 : 0;
         }
+    // a block needs masking when it reaches past the lowest position or
+    // starts below the highest window start of the CTA's rows
+    int min_pos = ctx - 1, max_lo = 0;
+    for (int tq = 0; tq < p.q_len; ++tq) {
+        const int ps = min(ctx - 1, query_position(p, b, ctx, tq));
+        min_pos = min(min_pos, ps);
+        if (p.window > 0)
+            max_lo = max(max_lo, ps - p.window + 1);
+    }
 
     float kfac = p.scale_log2;
-    if constexpr (KVT == kKvFp8)
-        kfac *= __ldg(p.k_scale + h);
+    if constexpr (kv_has_head_scale(KVT))
+        kfac *= __ldg(p.k_scale + h * p.scale_stride);
 
     float o[NT][8][4];
     float m[NT][2], l[NT][2];
@@ -355,6 +551,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
             uint8_t *dst = my_tiles + stage * C::kStageBytes;
             tma_tile_2d_g2s(dst, &kmap, 0, y, bar);
             tma_tile_2d_g2s(dst + C::kTileBytes, &vmap, 0, y, bar);
+            if constexpr (KVT == kKvFp16) {   // second 128-byte half of each row
+                tma_tile_2d_g2s(dst + BS * 128, &kmap, 128, y, bar);
+                tma_tile_2d_g2s(dst + C::kTileBytes + BS * 128, &vmap, 128, y, bar);
+            }
             if constexpr (KVT == kKvInt8) {
                 uint16_t *sd = my_scales + stage * C::kScaleHalves;
                 tma_bulk_g2s(sd, p.k_scale_tok + (size_t)y, BS * 2, bar);
@@ -367,7 +567,6 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     for (; issued < S && issued < n_it; ++issued)
         issue(issued);
 
-    const int min_pos = ctx - p.q_len;
     int it = 0;
     bool ok = true;
     for (; it < n_it; it += U) {
@@ -390,9 +589,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
             const uint8_t *kt = my_tiles + stage * C::kStageBytes;
             const uint16_t *st = my_scales + stage * C::kScaleHalves;
             if (have[u]) {
-                qk_block<KVT, NT, MT>(kt, st, g, t, qf, kfac, sc[u]);
+                if constexpr (KVT == kKvFp16)
+                    qk_block_f16<NT, MT, BS>(kt, g, t, qf, kfac, sc[u]);
+                else
+                    qk_block<KVT, NT, MT>(kt, st, g, t, qf, kfac, sc[u]);
                 const int key0 = lblk(it + u) * BS;
-                if (key0 + BS - 1 > min_pos) {   // a key may lie past a row's position
+                // a key may lie past a row's position or below its window
+                if (key0 + BS - 1 > min_pos || key0 < max_lo) {
 #pragma unroll
                     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -400,7 +603,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
                             for (int c = 0; c < 4; ++c) {
                                 const int key = key0 + mt * 16 + g + (c >> 1) * 8;
-                                if (key > pos[nt][c & 1])
+                                if (key > pos[nt][c & 1] || key < lo[nt][c & 1])
                                     sc[u][mt][nt][c] = -INFINITY;
                             }
                 }
@@ -464,7 +667,10 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
             const int stage = (it + u) % S;
             const uint8_t *vt = my_tiles + stage * C::kStageBytes + C::kTileBytes;
             const uint16_t *st = my_scales + stage * C::kScaleHalves;
-            pv_block<KVT, NT, MT, BS>(vt, st, g, t, lblk(it + u) * BS, ctx, sc[u], o);
+            if constexpr (KVT == kKvFp16)
+                pv_block_f16<NT, MT, BS>(vt, g, t, lblk(it + u) * BS, ctx, sc[u], o);
+            else
+                pv_block<KVT, NT, MT, BS>(vt, st, g, t, lblk(it + u) * BS, ctx, sc[u], o);
         }
 
         __syncwarp();
@@ -525,8 +731,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 
     const int d = threadIdx.x;   // 128 threads <-> 128 dims
     float vfac = 1.0f;
-    if constexpr (KVT == kKvFp8)
-        vfac = __ldg(p.v_scale + h);
+    if constexpr (kv_has_head_scale(KVT))
+        vfac = __ldg(p.v_scale + h * p.scale_stride);
     // Rows are independent: the loop is unrolled so that their shared-memory
     // reads and global stores overlap.
 #pragma unroll 4
@@ -559,17 +765,41 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
                 *reinterpret_cast<float2 *>(p.ws_ml + wrow * 2) = make_float2(M, L);
         }
     }
+    if (si.nsplit == 1 || !p.ws_cnt)
+        return;
+    // The last CTA of this (row group, KV head, sequence) to finish merges its
+    // splits: each CTA publishes its partial (fence), then counts itself in;
+    // the one that completes the count resets it for the next call and reads
+    // every partial.
+    __threadfence();
+    __syncthreads();
+    int *last = reinterpret_cast<int *>(smem);   // the tiles are idle now
+    if (threadIdx.x == 0) {
+        int *cnt = p.ws_cnt + (size_t)blockIdx.y * p.num_splits + si.first;
+        const int done = atomicAdd(cnt, 1) + 1;
+        *last = done >= si.nsplit;
+        if (done >= si.nsplit)
+            atomicExch(cnt, 0);
+    }
+    __syncthreads();
+    if (!*last)
+        return;
+    __threadfence();
+    // warp w merges rows w, w + 4, ... of this CTA's row group
+    for (int r = warp; r < RC; r += kWarps) {
+        const int rr = rg * RC + r;
+        if (rr >= p.rows)
+            break;
+        MergeRow mr;
+        mr.row0 = (size_t)blockIdx.y * p.num_splits * RC + r;
+        mr.stride = RC;
+        mr.load(p, si.first, si.nsplit, 0, lane);
+        mr.finish(p, si.first, si.nsplit, b, h, rr, lane);
+    }
 }
 
-// Merge of the split partial states (one warp per output row):
-// M = max_i m_i, L = sum_i l_i 2^(m_i - M), O = sum_i O_i 2^(m_i - M) / L.
-// The splits are taken kMergeChunk at a time: every lane issues the loads of
-// a whole chunk (the (m, l) pairs, the same for all lanes, and its float4 of
-// each O row) before using any, so a chunk costs one memory round trip; the
-// chunks are combined online.  A sequence that a single split covered was
-// finished by that split.
-constexpr int kMergeChunk = 16;
-
+// Merge of the split partial states by a separate kernel (the tensor-core
+// decode kernels' partials), one warp per output row.
 template <int BS>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
 {
@@ -582,74 +812,29 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
     const int rr = (int)(gw % p.rows);
     const int h = (int)((gw / p.rows) % p.num_kv_heads);
     const int b = (int)(gw / ((long long)p.rows * p.num_kv_heads));
-    const float vfac = p.v_scale ? __ldg(p.v_scale + h) : 1.0f;
     // slots first .. first + nsplit - 1 of unit (row group, KV head) y
     const int y = (rr / p.rows_per_cta) * p.num_kv_heads + h;
-    const size_t row0 = (size_t)y * p.num_splits * p.rows_per_cta + rr % p.rows_per_cta;
-    const size_t stride = p.rows_per_cta;
-    float2 ml[kMergeChunk];
-    float4 v[kMergeChunk];
-    auto load_chunk = [&](int first, int nsplit, int s0) {
-#pragma unroll
-        for (int k = 0; k < kMergeChunk; ++k) {
-            ml[k] = make_float2(-INFINITY, 0.0f);
-            v[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (s0 + k < nsplit && first + s0 + k < p.num_splits) {
-                const size_t wrow = row0 + (size_t)(first + s0 + k) * stride;
-                ml[k] = *reinterpret_cast<const float2 *>(p.ws_ml + wrow * 2);
-                v[k] = reinterpret_cast<const float4 *>(p.ws_o + wrow * kHeadDim)[lane];
-            }
-        }
-    };
+    MergeRow mr;
+    mr.row0 = (size_t)y * p.num_splits * p.rows_per_cta + rr % p.rows_per_cta;
+    mr.stride = p.rows_per_cta;
     // The first chunk is loaded for the slots all sequences at
     // max_context_len would give, while the real slots are computed from the
     // context lengths; it is reloaded only when they differ.
     const int gfirst = b * p.uniform_splits;
-    load_chunk(gfirst, p.uniform_splits, 0);
+    mr.load(p, gfirst, p.uniform_splits, 0, lane);
     const SplitInfo si = find_split<BS>(p, -1, b);
     if (si.nsplit <= 1)
         return;   // a single split wrote the final row itself
     if (si.first != gfirst || si.nsplit != p.uniform_splits)
-        load_chunk(si.first, si.nsplit, 0);
-    const int nvalid = si.nsplit;
-    float M = -INFINITY, L = 0.0f;
-    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < nvalid; s0 += kMergeChunk) {
-        if (s0 > 0)
-            load_chunk(si.first, nvalid, s0);
-        float cm = M;
-#pragma unroll
-        for (int k = 0; k < kMergeChunk; ++k)
-            cm = fmaxf(cm, ml[k].x);
-        const float mu = cm == -INFINITY ? 0.0f : cm;
-        const float corr = fast_exp2(M - mu);
-        L *= corr;
-        O.x *= corr, O.y *= corr, O.z *= corr, O.w *= corr;
-#pragma unroll
-        for (int k = 0; k < kMergeChunk; ++k) {
-            const float e = fast_exp2(ml[k].x - mu);
-            L += ml[k].y * e;
-            O.x += v[k].x * e, O.y += v[k].y * e, O.z += v[k].z * e, O.w += v[k].w * e;
-        }
-        M = cm;
-    }
-    const int tq = rr / p.group, gq = rr % p.group;
-    const size_t orow = ((size_t)b * p.q_len + tq) * p.num_q_heads + h * p.group + gq;
-    __half2 lo = __floats2half2_rn(L > 0.0f ? O.x / L * vfac : 0.0f, L > 0.0f ? O.y / L * vfac : 0.0f);
-    __half2 hi = __floats2half2_rn(L > 0.0f ? O.z / L * vfac : 0.0f, L > 0.0f ? O.w / L * vfac : 0.0f);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t *>(&lo);
-    pk.y = *reinterpret_cast<uint32_t *>(&hi);
-    reinterpret_cast<uint2 *>(p.out + orow * kHeadDim)[lane] = pk;
-    if (lane == 0 && p.lse)
-        p.lse[orow] = L > 0.0f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        mr.load(p, si.first, si.nsplit, 0, lane);
+    mr.finish(p, si.first, si.nsplit, b, h, rr, lane);
 }
 
 template <int KVT, int NT, int BS>
 cudaError_t launch_split(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                          cudaStream_t stream)
 {
-    constexpr size_t smem = decode_smem_bytes<BS>();
+    constexpr size_t smem = decode_smem_bytes<KVT, BS>();
     auto kern = decode_split_kernel<KVT, NT, BS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
@@ -683,7 +868,7 @@ template <int KVT, int NT, int BS>
 int occupancy_of()
 {
     auto kern = decode_split_kernel<KVT, NT, BS>;
-    constexpr size_t smem = decode_smem_bytes<BS>();
+    constexpr size_t smem = decode_smem_bytes<KVT, BS>();
     int n = 0;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
             cudaSuccess ||
@@ -705,21 +890,30 @@ int occupancy_bs(int block_size)
 
 // Resident split CTAs per SM for one kernel instance (registers and shared
 // memory decide it), cached per device; 2 where it cannot be queried.
+template <int KVT>
+int occupancy_nt(int nt, int block_size)
+{
+    return nt == 1 ? occupancy_bs<KVT, 1>(block_size) : occupancy_bs<KVT, 2>(block_size);
+}
+
 int split_occupancy(int kv_dtype, int nt, int block_size)
 {
     constexpr int kMaxDev = 64;
-    static int cache[kMaxDev][2][2][3] = {};
+    static int cache[kMaxDev][4][2][3] = {};
     int dev = 0;
     const int bi = block_size == 16 ? 0 : (block_size == 32 ? 1 : 2);
-    const int di = kv_dtype == kKvFp8 ? 0 : 1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+    if (kv_dtype < 0 || kv_dtype > 3 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 ||
+        dev >= kMaxDev)
         return 2;
-    int &c = cache[dev][di][nt - 1][bi];
+    int &c = cache[dev][kv_dtype][nt - 1][bi];
     if (!c) {
-        int n = di == 0 ? (nt == 1 ? occupancy_bs<kKvFp8, 1>(block_size)
-                                   : occupancy_bs<kKvFp8, 2>(block_size))
-                        : (nt == 1 ? occupancy_bs<kKvInt8, 1>(block_size)
-                                   : occupancy_bs<kKvInt8, 2>(block_size));
+        int n = 0;
+        switch (kv_dtype) {
+        case kKvFp8: n = occupancy_nt<kKvFp8>(nt, block_size); break;
+        case kKvInt8: n = occupancy_nt<kKvInt8>(nt, block_size); break;
+        case kKvE5m2: n = occupancy_nt<kKvE5m2>(nt, block_size); break;
+        default: n = occupancy_nt<kKvFp16>(nt, block_size); break;
+        }
         c = n > 0 ? n : 2;
     }
     return c;
@@ -738,16 +932,21 @@ bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv
     // CTA for all rows, so every code is fetched and converted once; the
     // mma.sync kernel would split the rows into groups that each convert it.
     plan->tc = rows > 16 && rows <= 128;
+    // up to 64 rows: keys on the tensor core's M and 128-key tiles, so that
+    // the softmax runs one thread per key instead of one per padded row
+    plan->tn = plan->tc && rows <= 64;
     plan->nt = plan->tc ? 0 : (rows <= 8 ? 1 : 2);
     plan->rows_per_cta = plan->tc ? rows : 8 * plan->nt;
     plan->row_groups = (rows + plan->rows_per_cta - 1) / plan->rows_per_cta;
     const int max_blocks = (max_context_len + block_size - 1) / block_size;
     const int units = num_kv_heads * plan->row_groups;   // grid y: (row group, KV head)
-    // splits: tensor-core kernel in whole 64-key tiles, at least 4 of them;
-    // mma.sync kernel at least kMinBlocksPerWarp blocks per warp
-    const int min_blocks = plan->tc ? 4 * (64 / block_size) : kWarps * kMinBlocksPerWarp;
+    // splits: tensor-core kernels in whole key tiles (64 keys with rows on M,
+    // 128 with keys on M), at least 256 keys; mma.sync kernel at least
+    // kMinBlocksPerWarp blocks per warp
+    const int tile_keys = plan->tn ? 128 : 64;
+    const int min_blocks = plan->tc ? 256 / block_size : kWarps * kMinBlocksPerWarp;
     plan->split_min_blocks = min_blocks;
-    plan->split_gran = plan->tc ? 64 / block_size : 1;
+    plan->split_gran = plan->tc ? tile_keys / block_size : 1;
     // C CTA slots per unit, at most `ctas_per_sm` CTAs on every SM (3, or
     // what fits), all resident in one wave, each slot given about the same
     // number of blocks on the device.  Rounding the count up instead would
@@ -775,9 +974,20 @@ bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv
     plan->uniform_bpc = split_blocks((long long)batch * max_blocks, (int)C, batch, max_blocks,
                                      plan->split_min_blocks, plan->split_gran);
     plan->uniform_splits = max(1, (max_blocks + plan->uniform_bpc - 1) / plan->uniform_bpc);
-    plan->workspace_bytes = C > batch ? (size_t)units * C * plan->rows_per_cta *
+    const size_t partials = C > batch ? (size_t)units * C * plan->rows_per_cta *
                                             (kHeadDim + 2) * sizeof(float)
                                       : 0;
+    // The mma.sync kernel merges its own splits, counting arrivals per
+    // (unit, sequence) at the sequence's first slot.  The counters sit in a
+    // leading area of fixed size for the device (units x C <= 16 CTAs per SM
+    // whenever C > batch), ahead of the partials of every plan, so that no
+    // call's partials ever land on them: they are zero between calls.
+    plan->fused_merge = partials > 0 && !plan->tc;
+    plan->counters_bytes =
+        partials > 0 ? ((size_t)16 * device_sm_count() * sizeof(int) + 255) / 256 * 256 : 0;
+    if (plan->fused_merge && (long long)units * C > 16LL * device_sm_count())
+        return false;
+    plan->workspace_bytes = plan->counters_bytes + partials;
     return true;
 }
 
@@ -785,16 +995,25 @@ cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_
                           const CUtensorMap &kmap, const CUtensorMap &vmap, cudaStream_t stream)
 {
     cudaError_t e;
-    if (plan.tc)
+    const bool one = plan.nt == 1;
+    if (plan.tn)
+        e = launch_decode_tn(p, kv_dtype, kmap, vmap, stream);
+    else if (plan.tc)
         e = launch_decode_tc(p, kv_dtype, kmap, vmap, stream);
     else if (kv_dtype == kKvFp8)
-        e = plan.nt == 1 ? launch_bs<kKvFp8, 1>(p, kmap, vmap, stream)
-                         : launch_bs<kKvFp8, 2>(p, kmap, vmap, stream);
+        e = one ? launch_bs<kKvFp8, 1>(p, kmap, vmap, stream)
+                : launch_bs<kKvFp8, 2>(p, kmap, vmap, stream);
+    else if (kv_dtype == kKvInt8)
+        e = one ? launch_bs<kKvInt8, 1>(p, kmap, vmap, stream)
+                : launch_bs<kKvInt8, 2>(p, kmap, vmap, stream);
+    else if (kv_dtype == kKvE5m2)
+        e = one ? launch_bs<kKvE5m2, 1>(p, kmap, vmap, stream)
+                : launch_bs<kKvE5m2, 2>(p, kmap, vmap, stream);
     else
-        e = plan.nt == 1 ? launch_bs<kKvInt8, 1>(p, kmap, vmap, stream)
-                         : launch_bs<kKvInt8, 2>(p, kmap, vmap, stream);
-    if (e != cudaSuccess || p.num_splits <= p.batch)
-        return e;   // one slot per sequence: every split wrote its final rows
+        e = one ? launch_bs<kKvFp16, 1>(p, kmap, vmap, stream)
+                : launch_bs<kKvFp16, 2>(p, kmap, vmap, stream);
+    if (e != cudaSuccess || p.num_splits <= p.batch || plan.fused_merge)
+        return e;   // one slot per sequence, or the split kernel merged its own splits
     const long long rows_total = (long long)p.batch * p.num_kv_heads * p.rows;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((rows_total + 3) / 4));

@@ -38,11 +38,18 @@
 // Epilogue: the final fp16 row when one split covers the sequence, otherwise
 // an FP32 partial (unnormalised O, max in log2 units, sum) in the decode
 // workspace, which the decode merge kernel combines.
+//
+// FP16 caches need no conversion: the TMA warp copies each block's two
+// 128-byte row halves straight into a K/V buffer (the same swizzled layout),
+// and the dequant warps only clear the rows past the context or the split
+// before releasing the buffer to the MMA warp (never-written slots may hold
+// NaN patterns, and 0 * NaN in P V would poison O).
 #include "common.cuh"
 #include "internal.h"
 #include "split_map.cuh"
 #include "tc.cuh"
 
+#include <climits>
 #include <math.h>
 
 namespace pkvq {
@@ -76,7 +83,7 @@ constexpr int kCodeStage = 16384;
 constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // stages x (K 64, V 64) halves
 constexpr int kOffKsf = kOffScl + kCodeStages * 256;            // bufs x 64 fp32 K factors
 constexpr int kOffBars = kOffKsf + kKVBufs * 64 * 4;
-constexpr int kNumBars = 1 + 2 * kCodeStages + 2 * kKVBufs + 3 * 2 + 1;
+constexpr int kNumBars = 1 + 2 * kCodeStages + 3 * kKVBufs + 3 * 2 + 1;
 constexpr int kOffTaddr = kOffBars + kNumBars * 8;
 constexpr int kSmemBytes = kOffTaddr + 16;
 constexpr size_t kSmemAlloc = kSmemBytes + 1024;
@@ -91,6 +98,7 @@ struct Bars {
     uint64_t *kv_full, *kv_empty;       // [kKVBufs]
     uint64_t *s_full, *p_full, *pv_done;   // [S/P buffer]
     uint64_t *mma_done;
+    uint64_t *kv_tma;                   // [kKVBufs] FP16: the buffer's copies landed
 };
 
 __device__ __forceinline__ Bars carve_bars(uint8_t *smem)
@@ -106,6 +114,7 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *smem)
     r.p_full = r.s_full + 2;
     r.pv_done = r.p_full + 2;
     r.mma_done = r.pv_done + 2;
+    r.kv_tma = r.mma_done + 1;
     return r;
 }
 
@@ -126,6 +135,8 @@ __device__ __forceinline__ void cvt4(uint32_t x, uint32_t &lo, uint32_t &hi)
 {
     if constexpr (KVT == kKvFp8)
         e4m3x4_to_half2x2(x, lo, hi);
+    else if constexpr (KVT == kKvE5m2)
+        e5m2x4_to_half2x2(x, lo, hi);
     else
         s8x4_to_half2x2(x, lo, hi);
 }
@@ -158,6 +169,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         for (int i = 0; i < kKVBufs; ++i) {
             mbar_init(&bars.kv_full[i], kDequantWarps);
             mbar_init(&bars.kv_empty[i], 1);
+            mbar_init(&bars.kv_tma[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars.s_full[i], 1);
@@ -179,7 +191,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     const int b = si.b;
     const int ctx = si.ctx;
     const int nblk_seq = (ctx + BS - 1) / BS;
-    const int blk_begin = si.split * si.bpc;   // a multiple of kBPT
+    const int blk_begin = si.blk0 + si.split * si.bpc;   // bpc is a multiple of kBPT
     const int blk_end = min(nblk_seq, blk_begin + si.bpc);
     const int nblk = max(0, blk_end - blk_begin);
     const int ntiles = (nblk + kBPT - 1) / kBPT;
@@ -205,10 +217,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         int win1 = 32 + lane < nwin ? __ldg(bt + 32 + lane) : 0;
         int wbase = 0;
         int issued = 0;
+        // FP16: each tile goes straight into K/V buffer j % kKVBufs
+        constexpr int kRing = KVT == kKvFp16 ? kKVBufs : kCodeStages;
         for (int j = 0; j < ntiles; ++j) {
-            const int s = j % kCodeStages;
-            if (j >= kCodeStages &&
-                !warp_wait(&bars.code_empty[s], ((j - kCodeStages) / kCodeStages) & 1, p.status))
+            const int s = j % kRing;
+            uint64_t *empty = KVT == kKvFp16 ? bars.kv_empty : bars.code_empty;
+            if (j >= kRing && !warp_wait(&empty[s], ((j - kRing) / kRing) & 1, p.status))
                 break;
             issued = j + 1;
             const int blk0 = j * kBPT;   // within this split
@@ -221,7 +235,30 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 const int c = __shfl_sync(0xffffffffu, win1, bi & 31);
                 ids[i] = (bi - wbase) < 32 ? a : c;
             }
-            if (lane == 0) {
+            if (KVT == kKvFp16 && lane == 0) {
+                mbar_arrive_expect_tx(&bars.kv_tma[s], (uint32_t)nb * BS * 256 * 2);
+                uint8_t *kv = smem + kOffKV + s * kKVBuf;
+#pragma unroll
+                for (int i = 0; i < kBPT; ++i) {
+                    if (i >= nb)
+                        break;
+                    int phys = ids[i];
+#ifdef PKVQ_BOUNDS_CHECK
+                    if (phys < 0 || phys >= p.num_blocks) {
+                        atomicOr(p.status, kStatusBadBlock);
+                        phys = 0;
+                    }
+#endif
+                    const int y = (phys * p.num_kv_heads + h) * BS;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        tma_tile_2d_g2s(kv + half * 8192 + i * BS * 128, &kmap, 128 * half, y,
+                                        &bars.kv_tma[s]);
+                        tma_tile_2d_g2s(kv + 16384 + half * 8192 + i * BS * 128, &vmap,
+                                        128 * half, y, &bars.kv_tma[s]);
+                    }
+                }
+            } else if (lane == 0) {
                 uint32_t tx = (uint32_t)nb * BS * 128 * 2;
                 if constexpr (KVT == kKvInt8)
                     tx += (uint32_t)nb * BS * 2 * 2;
@@ -257,9 +294,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             }
         }
         // copies this CTA issued must land before it exits (bounded wait)
-        if (lane == 0)
-            for (int j = max(0, issued - kCodeStages); j < issued; ++j)
-                mbar_wait(&bars.code_full[j % kCodeStages], (j / kCodeStages) & 1, nullptr);
+        if (lane == 0) {
+            uint64_t *full = KVT == kKvFp16 ? bars.kv_tma : bars.code_full;
+            for (int j = max(0, issued - kRing); j < issued; ++j)
+                mbar_wait(&full[j % kRing], (j / kRing) & 1, nullptr);
+        }
     } else if (warp == kWarpMma) {
         // --------------------------------------------------- MMA issuer --
         // S(k) overwrites P(k-2) in the same buffer, so Q K(k)^T is issued
@@ -337,7 +376,34 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         const int c0 = warp >= 6 ? 4 : 0;         // first 16-byte chunk of the row
         const int nch = isv ? 8 : 4;              // chunks this warp converts
         const float kfac = p.scale_log2;
-        for (int j = 0; j < ntiles; ++j) {
+        if constexpr (KVT == kKvFp16) {
+            // clear the rows no key of this split may read, then release
+            for (int j = 0; j < ntiles; ++j) {
+                const int bj = j % kKVBufs;
+                if (!warp_wait(&bars.kv_tma[bj], (j / kKVBufs) & 1, p.status))
+                    break;
+                const int key = key_begin + j * kKT + row;
+                if (key >= ctx || j * kKT + row >= nblk * BS) {
+                    // the whole 128-byte row of each d half this warp owns
+                    // (K: half c0 / 4; V: both)
+                    uint8_t *kv = smem + kOffKV + bj * kKVBuf + isv * 16384;
+                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        if (!isv && hh != (c0 >> 2))
+                            continue;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<uint4 *>(kv + hh * 8192 + row * 128 + c * 16) = z;
+                    }
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars.kv_full[bj]);
+            }
+        }
+        for (int j = 0; KVT != kKvFp16 && j < ntiles; ++j) {
             const int s = j % kCodeStages, bj = j % kKVBufs;
             if (!warp_wait(&bars.code_full[s], (j / kCodeStages) & 1, p.status))
                 break;
@@ -413,8 +479,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         const uint32_t tl = tmem + ((uint32_t)(32 * sw) << 16);
         const int tq = r / G, gq = r % G;
         const bool valid = r < p.rows;
-        const int pos = ctx - p.q_len + tq;   // keys 0..pos are visible to this row
-        const int pos_lo = ctx - p.q_len;     // the first row's position
+        // keys lo..pos are visible to this row (padding rows: the whole split)
+        const int pos = valid ? min(ctx - 1, query_position(p, b, ctx, tq)) : ctx - 1;
+        const int lo = p.window > 0 && valid ? pos - p.window + 1 : INT_MIN;
+        // a tile needs masking when it reaches past the lowest position or
+        // starts below the highest window start of the rows
+        int pos_lo = ctx - 1, lo_hi = INT_MIN;
+        for (int t = 0; t < p.q_len; ++t) {
+            const int ps = min(ctx - 1, query_position(p, b, ctx, t));
+            pos_lo = min(pos_lo, ps);
+            if (p.window > 0)
+                lo_hi = max(lo_hi, ps - p.window + 1);
+        }
         const size_t qrow = ((size_t)b * p.q_len + tq) * p.num_q_heads + (size_t)h * G + gq;
 
         // Q row -> tensor memory (two fp16 per column), zeros for padding rows
@@ -438,8 +514,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         }
 
         float kfac = p.scale_log2;
-        if constexpr (KVT == kKvFp8)
-            kfac *= __ldg(p.k_scale + h);
+        if constexpr (kv_has_head_scale(KVT))
+            kfac *= __ldg(p.k_scale + h * p.scale_stride);
         float m_used = -INFINITY, l = 0.0f;
         bool ok = true;
         for (int j = 0; j < ntiles; ++j) {
@@ -466,7 +542,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 }
             }
             const int key0 = key_begin + j * kKT;
-            if constexpr (KVT == kKvFp8) {
+            if constexpr (KVT != kKvInt8) {
                 const float2 f2 = make_float2(kfac, kfac);
 #pragma unroll
                 for (int c = 0; c < kKT; c += 2) {
@@ -487,10 +563,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             // split are masked; only tiles that reach past the first row's
             // position or the split's end need it
             const int key_lim = key_begin + nblk * BS;   // first key past the split
-            if (key0 + kKT - 1 > pos_lo || key0 + kKT > key_lim) {
+            if (key0 + kKT - 1 > pos_lo || key0 + kKT > key_lim || key0 < lo_hi) {
 #pragma unroll
                 for (int c = 0; c < kKT; ++c)
-                    if (key0 + c > pos || key0 + c >= key_lim)
+                    if (key0 + c > pos || key0 + c >= key_lim || key0 + c < lo)
                         v[c] = -INFINITY;
             }
             float m8[8];
@@ -561,8 +637,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             tc_fence_after();
         if (si.nsplit == 1) {
             float vfac = 1.0f;
-            if constexpr (KVT == kKvFp8)
-                vfac = __ldg(p.v_scale + h);
+            if constexpr (kv_has_head_scale(KVT))
+                vfac = __ldg(p.v_scale + h * p.scale_stride);
             const float f = (have_o && l > 0.0f) ? vfac / l : 0.0f;
             __half *dst = p.out + qrow * kHeadDim;
 #pragma unroll
@@ -647,14 +723,14 @@ cudaError_t launch_tc(const DecodeParams &p, const CUtensorMap &kmap, const CUte
 cudaError_t launch_decode_tc(const DecodeParams &p, int kv_dtype, const CUtensorMap &kmap,
                              const CUtensorMap &vmap, cudaStream_t stream)
 {
-    const bool fp8 = kv_dtype == kKvFp8;
-    switch (p.block_size) {
-    case 16: return fp8 ? launch_tc<kKvFp8, 16>(p, kmap, vmap, stream)
-                        : launch_tc<kKvInt8, 16>(p, kmap, vmap, stream);
-    case 32: return fp8 ? launch_tc<kKvFp8, 32>(p, kmap, vmap, stream)
-                        : launch_tc<kKvInt8, 32>(p, kmap, vmap, stream);
-    case 64: return fp8 ? launch_tc<kKvFp8, 64>(p, kmap, vmap, stream)
-                        : launch_tc<kKvInt8, 64>(p, kmap, vmap, stream);
+    switch (kv_dtype * 100 + p.block_size) {
+#define PKVQ_TC_CASE(T, B) \
+    case T * 100 + B: return launch_tc<T, B>(p, kmap, vmap, stream);
+        PKVQ_TC_CASE(kKvFp8, 16) PKVQ_TC_CASE(kKvFp8, 32) PKVQ_TC_CASE(kKvFp8, 64)
+        PKVQ_TC_CASE(kKvInt8, 16) PKVQ_TC_CASE(kKvInt8, 32) PKVQ_TC_CASE(kKvInt8, 64)
+        PKVQ_TC_CASE(kKvE5m2, 16) PKVQ_TC_CASE(kKvE5m2, 32) PKVQ_TC_CASE(kKvE5m2, 64)
+        PKVQ_TC_CASE(kKvFp16, 16) PKVQ_TC_CASE(kKvFp16, 32) PKVQ_TC_CASE(kKvFp16, 64)
+#undef PKVQ_TC_CASE
     default: return cudaErrorInvalidValue;
     }
 }

@@ -10,13 +10,24 @@
 
 namespace pkvq {
 
-constexpr int kKvFp8 = 0;
+constexpr int kKvFp8 = 0;     // E4M3
 constexpr int kKvInt8 = 1;
+constexpr int kKvE5m2 = 2;
+constexpr int kKvFp16 = 3;
 constexpr int kHeadDim = 128;
+
+// Bytes per stored cache element of a format.
+__host__ __device__ constexpr int kv_elem_bytes(int kvt) { return kvt == kKvFp16 ? 2 : 1; }
+// Formats with a static fp32 scale per KV head (or per layer).
+__host__ __device__ constexpr bool kv_has_head_scale(int kvt)
+{
+    return kvt == kKvFp8 || kvt == kKvE5m2;
+}
 
 struct KvWriteParams {
     uint8_t *k_cache, *v_cache;
-    const float *k_scale, *v_scale;        // FP8
+    const float *k_scale, *v_scale;        // FP8 formats
+    int scale_stride;                      // 1: per KV head; 0: one scale per layer
     uint16_t *k_scale_tok, *v_scale_tok;   // INT8 (fp16 bits)
     const __half *k, *v;
     const int32_t *slot_mapping;
@@ -27,8 +38,11 @@ struct KvWriteParams {
 cudaError_t launch_kv_write_quant(const KvWriteParams &p, int kv_dtype, cudaStream_t stream);
 
 struct DecodeParams {
-    const float *k_scale, *v_scale;              // FP8: per KV head
+    const float *k_scale, *v_scale;              // FP8 formats: per KV head (or layer)
+    int scale_stride;                            // 1: per KV head; 0: one per layer
     const uint16_t *k_scale_tok, *v_scale_tok;   // INT8: per (block, head, token)
+    int window;                                  // > 0: sliding window of keys
+    const int32_t *query_pos;                    // nullable [batch][q_len]
     const __half *q;
     __half *out;
     float *lse;
@@ -47,6 +61,9 @@ struct DecodeParams {
     float scale_log2;    // softmax_scale * log2(e)
     float *ws_o;         // [row groups x Hkv][C][rows_per_cta][128] fp32, unnormalised
     float *ws_ml;        // [row groups x Hkv][C][rows_per_cta][2] fp32 (log2 max, sum)
+    int *ws_cnt;         // arrival counters [row groups x Hkv][C] (at the first slot of
+                         // each sequence), or null: the split kernel's last CTA of a
+                         // sequence merges it; zero between calls
     uint32_t *status;
 };
 
@@ -57,6 +74,9 @@ struct DecodePlan {
     int uniform_splits, uniform_bpc;    // the assignment with equal lengths
     int split_min_blocks, split_gran;
     bool tc;                            // tensor-core kernel: all rows of a KV head in one CTA
+    bool tn;                            // ... with keys on M (17..64 rows), else rows on M
+    bool fused_merge;                   // the mma.sync kernel merges its own splits
+    size_t counters_bytes;              // the workspace's leading counter area
     size_t workspace_bytes;
 };
 
@@ -65,8 +85,11 @@ struct DecodePlan {
 bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv_heads,
                  int block_size, int max_context_len, DecodePlan *plan);
 
-// The tensor-core decode kernel (all rows of a KV head in one CTA).
+// The tensor-core decode kernels (all rows of a KV head in one CTA): query
+// rows on the MMA's M (65..128 rows) or keys on M (17..64 rows).
 cudaError_t launch_decode_tc(const DecodeParams &p, int kv_dtype, const CUtensorMap &kmap,
+                             const CUtensorMap &vmap, cudaStream_t stream);
+cudaError_t launch_decode_tn(const DecodeParams &p, int kv_dtype, const CUtensorMap &kmap,
                              const CUtensorMap &vmap, cudaStream_t stream);
 
 cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_dtype,
@@ -75,7 +98,9 @@ cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_
 
 struct PrefillParams {
     const float *k_scale, *v_scale;
+    int scale_stride;                            // 1: per KV head; 0: one per layer
     const uint16_t *k_scale_tok, *v_scale_tok;
+    int window;                                  // > 0: sliding window of keys
     const __half *q;
     __half *out;
     float *lse;
@@ -93,9 +118,36 @@ struct PrefillParams {
 cudaError_t launch_prefill_tc(const PrefillParams &p, int kv_dtype, const CUtensorMap &kmap,
                               const CUtensorMap &vmap, cudaStream_t stream);
 
-// Encodes a 2-D uint8 tensor map over a cache: rows of 128 bytes, boxes of
-// box_rows rows, 128-byte swizzle.
-bool make_cache_tensor_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows);
+// Encodes a 2-D uint8 tensor map over a cache: rows of row_bytes (128 or
+// 256) bytes, boxes of 128 bytes x box_rows rows, 128-byte swizzle.
+bool make_cache_tensor_map(CUtensorMap *map, const void *base, uint64_t rows, int box_rows,
+                           int row_bytes);
+
+struct MergeParams {
+    const __half *parts_out;   // [parts][rows][128]
+    const float *parts_lse;    // [parts][rows]
+    __half *out;
+    float *lse;
+    int parts;
+    long long rows;
+};
+
+cudaError_t launch_merge_states(const MergeParams &p, cudaStream_t stream);
+
+struct CopyParams {
+    const uint8_t *src_k, *src_v;
+    uint8_t *dst_k, *dst_v;
+    const uint16_t *src_ks, *src_vs;   // INT8 scales (or null)
+    uint16_t *dst_ks, *dst_vs;
+    const int32_t *pairs;
+    int n;
+    long long block_bytes;             // elements of one block (all heads), bytes
+    int block_scales;                  // INT8 scales of one block (all heads)
+    int src_blocks, dst_blocks;
+    uint32_t *status;
+};
+
+cudaError_t launch_copy_blocks(const CopyParams &p, cudaStream_t stream);
 
 int device_sm_count();
 

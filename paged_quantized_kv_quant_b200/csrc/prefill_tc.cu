@@ -34,10 +34,18 @@
 //               TMEM only when the row maximum grew by more than 2^8.  The
 //               tensor core runs one group's products while the other group's
 //               softmax runs.
+//
+// FP16 caches need no conversion: the TMA warp copies each block's two
+// 128-byte row halves straight into a K/V buffer, and the dequant warps only
+// clear rows past the context.  With a sliding window w ("1Cat-LLM" README,
+// "DFlash2 Long-Context Decay") the key loop starts at the tile holding the
+// window start of the CTA's first row, and rows mask keys below their own
+// window start.
 #include "common.cuh"
 #include "internal.h"
 #include "tc.cuh"
 
+#include <climits>
 #include <math.h>
 
 namespace pkvq {
@@ -65,7 +73,7 @@ constexpr int kCodeStage = 16384;
 constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // stages x (K 64, V 64) halves
 constexpr int kOffKsf = kOffScl + kCodeStages * 256;            // bufs x 64 fp32 K factors
 constexpr int kOffBars = kOffKsf + kKVBufs * 64 * 4;
-constexpr int kNumBars = 1 + 2 * kCodeStages + 2 * kKVBufs + 3 * 2 + 1;
+constexpr int kNumBars = 1 + 2 * kCodeStages + 3 * kKVBufs + 3 * 2 + 1;
 constexpr int kOffTaddr = kOffBars + kNumBars * 8;
 constexpr int kSmemBytes = kOffTaddr + 16;
 constexpr size_t kSmemAlloc = kSmemBytes + 1024;
@@ -80,6 +88,7 @@ struct Bars {
     uint64_t *kv_full, *kv_empty;       // [kKVBufs]
     uint64_t *s_full, *p_full, *pv_done;   // [tile]
     uint64_t *mma_done;                 // all MMAs retired (before TMEM is freed)
+    uint64_t *kv_tma;                   // [kKVBufs] FP16: the buffer's copies landed
 };
 
 __device__ __forceinline__ Bars carve_bars(uint8_t *smem)
@@ -95,6 +104,7 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *smem)
     r.p_full = r.s_full + 2;
     r.pv_done = r.p_full + 2;
     r.mma_done = r.pv_done + 2;
+    r.kv_tma = r.mma_done + 1;
     return r;
 }
 
@@ -117,6 +127,8 @@ __device__ __forceinline__ void cvt4(uint32_t x, uint32_t &lo, uint32_t &hi)
 {
     if constexpr (KVT == kKvFp8)
         e4m3x4_to_half2x2(x, lo, hi);
+    else if constexpr (KVT == kKvE5m2)
+        e5m2x4_to_half2x2(x, lo, hi);
     else
         s8x4_to_half2x2(x, lo, hi);
 }
@@ -125,19 +137,24 @@ __device__ __forceinline__ void cvt4(uint32_t x, uint32_t &lo, uint32_t &hi)
 struct QTile {
     int q0;        // first query token (within the sequence)
     int pos_lo;    // position of its first token
-    int ntiles;    // key tiles it needs (0: tile absent or sees no key)
+    int pos_hi;    // position of its last token
+    int ntiles;    // key tiles it needs from the CTA's first tile jbase on
+                   // (0: tile absent or sees no key)
 };
 
-__device__ __forceinline__ QTile make_qtile(int tile, int tokens_per_tile, int q_len, int ctx)
+__device__ __forceinline__ QTile make_qtile(int tile, int tokens_per_tile, int q_len, int ctx,
+                                            int jbase)
 {
     QTile t;
     t.q0 = tile * tokens_per_tile;
     t.pos_lo = ctx - q_len + t.q0;
+    t.pos_hi = t.pos_lo;
     t.ntiles = 0;
     if (t.q0 < q_len) {
         const int tq_end = min(q_len, t.q0 + tokens_per_tile);
+        t.pos_hi = ctx - q_len + tq_end - 1;
         const int nkeys = max(0, min(ctx, ctx - q_len + tq_end));
-        t.ntiles = (nkeys + kKT - 1) / kKT;
+        t.ntiles = max(0, (nkeys + kKT - 1) / kKT - jbase);
     }
     return t;
 }
@@ -165,10 +182,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         return;
     const int ctx = p.context_lens[b];
     const int G = p.group;
-    const QTile qt[2] = {make_qtile(2 * pair, p.tokens_per_tile, q_len, ctx),
-                         make_qtile(2 * pair + 1, p.tokens_per_tile, q_len, ctx)};
-    const int ntiles = max(qt[0].ntiles, qt[1].ntiles);
+    // first key tile any row of the CTA sees (tile A holds the lower positions)
+    const int jbase =
+        p.window > 0 ? max(0, ctx - q_len + 2 * pair * p.tokens_per_tile - p.window + 1) / kKT : 0;
+    const QTile qt[2] = {make_qtile(2 * pair, p.tokens_per_tile, q_len, ctx, jbase),
+                         make_qtile(2 * pair + 1, p.tokens_per_tile, q_len, ctx, jbase)};
+    const int ntiles = max(qt[0].ntiles, qt[1].ntiles);   // counted from jbase
     const int nblk_seq = (ctx + BS - 1) / BS;
+    const int blk_base = jbase * kBPT;                    // first block read
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -181,6 +202,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         for (int i = 0; i < kKVBufs; ++i) {
             mbar_init(&bars.kv_full[i], kDequantWarps);
             mbar_init(&bars.kv_empty[i], 1);
+            mbar_init(&bars.kv_tma[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars.s_full[i], 1);
@@ -205,22 +227,25 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             prefetch_tmap(&kmap);
             prefetch_tmap(&vmap);
         }
-        const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq;
+        const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq + blk_base;
         // every index stays inside the table row, even for a context longer
         // than the row can address (a caller error: those keys read block 0)
-        const int nblk_used = min(min(nblk_seq, ntiles * kBPT), p.max_blocks_per_seq);
+        const int nblk_used =
+            min(min(nblk_seq - blk_base, ntiles * kBPT), p.max_blocks_per_seq - blk_base);
         int win0 = lane < nblk_used ? __ldg(bt + lane) : 0;
         int win1 = 32 + lane < nblk_used ? __ldg(bt + 32 + lane) : 0;
         int wbase = 0;
         int issued = 0;
+        // FP16: each tile goes straight into K/V buffer j % kKVBufs
+        constexpr int kRing = KVT == kKvFp16 ? kKVBufs : kCodeStages;
         for (int j = 0; j < ntiles; ++j) {
-            const int s = j % kCodeStages;
-            if (j >= kCodeStages &&
-                !warp_wait(&bars.code_empty[s], ((j - kCodeStages) / kCodeStages) & 1, p.status))
+            const int s = j % kRing;
+            uint64_t *empty = KVT == kKvFp16 ? bars.kv_empty : bars.code_empty;
+            if (j >= kRing && !warp_wait(&empty[s], ((j - kRing) / kRing) & 1, p.status))
                 break;
             issued = j + 1;
-            const int blk0 = j * kBPT;
-            const int nb = min(kBPT, nblk_seq - blk0);
+            const int blk0 = j * kBPT;   // from blk_base
+            const int nb = min(kBPT, nblk_seq - blk_base - blk0);
             int ids[kBPT];
 #pragma unroll
             for (int i = 0; i < kBPT; ++i) {
@@ -229,7 +254,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 const int c = __shfl_sync(0xffffffffu, win1, bi & 31);
                 ids[i] = (bi - wbase) < 32 ? a : c;
             }
-            if (lane == 0) {
+            if (KVT == kKvFp16 && lane == 0) {
+                mbar_arrive_expect_tx(&bars.kv_tma[s], (uint32_t)nb * BS * 256 * 2);
+                uint8_t *kv = smem + kOffKV + s * kKVBuf;
+#pragma unroll
+                for (int i = 0; i < kBPT; ++i) {
+                    if (i >= nb)
+                        break;
+                    int phys = ids[i];
+#ifdef PKVQ_BOUNDS_CHECK
+                    if (phys < 0 || phys >= p.num_blocks) {
+                        atomicOr(p.status, kStatusBadBlock);
+                        phys = 0;
+                    }
+#endif
+                    const int y = (phys * p.num_kv_heads + h) * BS;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        tma_tile_2d_g2s(kv + half * 8192 + i * BS * 128, &kmap, 128 * half, y,
+                                        &bars.kv_tma[s]);
+                        tma_tile_2d_g2s(kv + 16384 + half * 8192 + i * BS * 128, &vmap,
+                                        128 * half, y, &bars.kv_tma[s]);
+                    }
+                }
+            } else if (lane == 0) {
                 uint32_t tx = (uint32_t)nb * BS * 128 * 2;
                 if constexpr (KVT == kKvInt8)
                     tx += (uint32_t)nb * BS * 2 * 2;
@@ -267,9 +315,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         // Copies this CTA issued must land before it exits: wait (bounded) for
         // the most recent round of every stage (already complete when the
         // consumers kept up).
-        if (lane == 0)
-            for (int j = max(0, issued - kCodeStages); j < issued; ++j)
-                mbar_wait(&bars.code_full[j % kCodeStages], (j / kCodeStages) & 1, nullptr);
+        if (lane == 0) {
+            uint64_t *full = KVT == kKvFp16 ? bars.kv_tma : bars.code_full;
+            for (int j = max(0, issued - kRing); j < issued; ++j)
+                mbar_wait(&full[j % kRing], (j / kRing) & 1, nullptr);
+        }
     } else if (warp == kWarpMma) {
         // --------------------------------------------------- MMA issuer --
         // Serves whichever query tile has its P ready (no head-of-line
@@ -375,7 +425,28 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         // ------------------------------------------------------ dequant --
         const int row = tid;   // 0..63: this thread converts key row `row` of K and V
         const float kfac = p.scale_log2;
-        for (int j = 0; j < ntiles; ++j) {
+        if constexpr (KVT == kKvFp16) {
+            // clear the rows past the context, then release the buffer
+            for (int j = 0; j < ntiles; ++j) {
+                const int bj = j % kKVBufs;
+                if (!warp_wait(&bars.kv_tma[bj], (j / kKVBufs) & 1, p.status))
+                    break;
+                if ((jbase + j) * kKT + row >= ctx) {
+                    uint8_t *kv = smem + kOffKV + bj * kKVBuf;
+                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int hh = 0; hh < 4; ++hh)   // K d halves 0, 1, V d halves 0, 1
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<uint4 *>(kv + hh * 8192 + row * 128 + c * 16) = z;
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&bars.kv_full[bj]);
+            }
+        }
+        for (int j = 0; KVT != kKvFp16 && j < ntiles; ++j) {
             const int s = j % kCodeStages, bj = j % kKVBufs;
             if (!warp_wait(&bars.code_full[s], (j / kCodeStages) & 1, p.status))
                 break;
@@ -385,7 +456,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             const uint8_t *codes = smem + kOffCodes + s * kCodeStage;
             const uint16_t *scl = reinterpret_cast<const uint16_t *>(smem + kOffScl + s * 256);
             uint8_t *kv = smem + kOffKV + bj * kKVBuf;
-            const int key0 = j * kKT;
+            const int key0 = (jbase + j) * kKT;
 #pragma unroll 4
             for (int k = 0; k < 16; ++k) {
                 const int isv = k >> 3;
@@ -465,8 +536,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         }
 
         float kfac = p.scale_log2;
-        if constexpr (KVT == kKvFp8)
-            kfac *= __ldg(p.k_scale + h);
+        if constexpr (kv_has_head_scale(KVT))
+            kfac *= __ldg(p.k_scale + h * p.scale_stride);
+        // keys lo..pos are visible to this row
+        const int lo = p.window > 0 ? pos - p.window + 1 : INT_MIN;
+        const int lo_hi = p.window > 0 ? T.pos_hi - p.window + 1 : INT_MIN;
         float m_used = -INFINITY, l = 0.0f;
         bool ok = true;
         for (int j = 0; j < T.ntiles; ++j) {
@@ -494,8 +568,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 }
             }
 
-            const int key0 = j * kKT;
-            if constexpr (KVT == kKvFp8) {
+            const int key0 = (jbase + j) * kKT;
+            if constexpr (KVT != kKvInt8) {
                 const float2 f2 = make_float2(kfac, kfac);
 #pragma unroll
                 for (int c = 0; c < kKT; c += 2) {
@@ -512,10 +586,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     v[c] = r2.x, v[c + 1] = r2.y;
                 }
             }
-            if (key0 + kKT - 1 > T.pos_lo) {   // a key may lie past a row's position
+            // a key may lie past a row's position or below its window
+            if (key0 + kKT - 1 > T.pos_lo || key0 < lo_hi) {
 #pragma unroll
                 for (int c = 0; c < kKT; ++c)
-                    if (key0 + c > pos)
+                    if (key0 + c > pos || key0 + c < lo)
                         v[c] = -INFINITY;
             }
             // row max: eight independent chains, then a tree
@@ -575,8 +650,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
 
         // ---- epilogue: O / l -> fp16 ----
         float vfac = 1.0f;
-        if constexpr (KVT == kKvFp8)
-            vfac = __ldg(p.v_scale + h);
+        if constexpr (kv_has_head_scale(KVT))
+            vfac = __ldg(p.v_scale + h * p.scale_stride);
         const bool have_o = ok && T.ntiles > 0 &&
                             warp_wait(&bars.pv_done[x], (T.ntiles - 1) & 1, p.status);
         if (have_o)
@@ -636,14 +711,14 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, int kv_dtype, const CUtens
 {
     if (p.q_tiles == 0 || p.batch == 0)
         return cudaSuccess;
-    const bool fp8 = kv_dtype == kKvFp8;
-    switch (p.block_size) {
-    case 16: return fp8 ? launch_tc<kKvFp8, 16>(p, kmap, vmap, stream)
-                        : launch_tc<kKvInt8, 16>(p, kmap, vmap, stream);
-    case 32: return fp8 ? launch_tc<kKvFp8, 32>(p, kmap, vmap, stream)
-                        : launch_tc<kKvInt8, 32>(p, kmap, vmap, stream);
-    case 64: return fp8 ? launch_tc<kKvFp8, 64>(p, kmap, vmap, stream)
-                        : launch_tc<kKvInt8, 64>(p, kmap, vmap, stream);
+    switch (kv_dtype * 100 + p.block_size) {
+#define PKVQ_TC_CASE(T, B) \
+    case T * 100 + B: return launch_tc<T, B>(p, kmap, vmap, stream);
+        PKVQ_TC_CASE(kKvFp8, 16) PKVQ_TC_CASE(kKvFp8, 32) PKVQ_TC_CASE(kKvFp8, 64)
+        PKVQ_TC_CASE(kKvInt8, 16) PKVQ_TC_CASE(kKvInt8, 32) PKVQ_TC_CASE(kKvInt8, 64)
+        PKVQ_TC_CASE(kKvE5m2, 16) PKVQ_TC_CASE(kKvE5m2, 32) PKVQ_TC_CASE(kKvE5m2, 64)
+        PKVQ_TC_CASE(kKvFp16, 16) PKVQ_TC_CASE(kKvFp16, 32) PKVQ_TC_CASE(kKvFp16, 64)
+#undef PKVQ_TC_CASE
     default: return cudaErrorInvalidValue;
     }
 }

@@ -5,10 +5,16 @@
 // slots.  The host knows only max_context_len; the context lengths live on
 // the device.  So each CTA maps its slot to a (sequence, split) pair itself:
 // sequence b gets nsplit_b = max(1, ceil(n_b / bpc)) consecutive slots, where
-// n_b is its number of cache blocks and bpc = split_blocks(...) below, which
-// keeps the total within C.  Sequences of different lengths then still give
-// every CTA about the same number of blocks.  The merge kernel recomputes
-// the same map to find a sequence's partials.
+// n_b is its number of cache blocks that any of its queries can see and
+// bpc = split_blocks(...) below, which keeps the total within C.  Sequences of
+// different lengths then still give every CTA about the same number of
+// blocks.  The merge kernel recomputes the same map to find a sequence's
+// partials.
+//
+// Visible blocks: a sequence's keys end at its context length; with a
+// sliding window w they start at the first query's position - w + 1 ("1Cat-LLM"
+// README, "DFlash2 Long-Context Decay": the paged loop starts at the window's
+// first tile), so blocks below it are neither read nor given a split.
 #pragma once
 
 #include "internal.h"
@@ -42,12 +48,36 @@ struct SplitInfo {
     int first;    // slot of its first split
     int ctx;      // its context length
     int bpc;      // blocks per split
+    int blk0;     // its first visible block (splits start at blk0 + split * bpc)
 };
 
+// Position of query token t of sequence b among the call's keys.
+__device__ __forceinline__ int query_position(const DecodeParams &p, int b, int ctx, int t)
+{
+    return p.query_pos ? p.query_pos[(size_t)b * p.q_len + t] : ctx - p.q_len + t;
+}
+
+// First block any query of sequence i can see (0 without a sliding window).
+template <int BS>
+__device__ __forceinline__ int seq_first_block(const DecodeParams &p, int i, int ctx)
+{
+    if (p.window <= 0)
+        return 0;
+    int lo = query_position(p, i, ctx, 0);
+    for (int t = 1; t < p.q_len; ++t)
+        lo = min(lo, query_position(p, i, ctx, t));
+    return max(0, lo - p.window + 1) / BS;
+}
+
+// Visible blocks of sequence i (0 for i >= batch).
 template <int BS>
 __device__ __forceinline__ int seq_blocks(const DecodeParams &p, int i)
 {
-    return i < p.batch ? (max(p.context_lens[i], 0) + BS - 1) / BS : 0;
+    if (i >= p.batch)
+        return 0;
+    const int ctx = max(p.context_lens[i], 0);
+    const int end = (ctx + BS - 1) / BS;
+    return max(0, end - seq_first_block<BS>(p, i, ctx));
 }
 
 // Computed by one whole warp (result warp-uniform).  slot >= 0: the
@@ -71,7 +101,8 @@ __device__ SplitInfo find_split(const DecodeParams &p, int slot, int seq)
     }
     SplitInfo r{-1, 0, 0, 0, 0,
                 split_blocks(total, p.num_splits, p.batch, longest, p.split_min_blocks,
-                             p.split_gran)};
+                             p.split_gran),
+                0};
     int run = 0;   // slots taken by the sequences before this chunk
     for (int base = 0; base < p.batch; base += 32) {
         const int i = base + lane;
@@ -95,6 +126,7 @@ __device__ SplitInfo find_split(const DecodeParams &p, int slot, int seq)
             r.nsplit = __shfl_sync(0xffffffffu, ns, src);
             r.split = slot >= 0 ? slot - r.first : 0;
             r.ctx = max(p.context_lens[r.b], 0);
+            r.blk0 = seq_first_block<BS>(p, r.b, r.ctx);
             break;
         }
         run += __shfl_sync(0xffffffffu, incl, 31);

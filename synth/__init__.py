@@ -245,3 +245,20 @@ def useful_flops(spec: CaseSpec) -> int:
         # query t sees c - ql + t + 1 keys
         pairs += ql * (c - ql) + ql * (ql + 1) // 2
     return 4 * spec.head_dim * spec.num_q_heads * pairs
+
+
+def attention_parts(parts: int, rows: int, head_dim: int = 128, seed: int = 0,
+                    empty_frac: float = 0.2):
+    """Per-part attention results over disjoint key sets, as the merge of a
+    sequence-sharded decode receives them: outputs fp16 [parts][rows][D]
+    ~ N(0,1), lse fp32 [parts][rows] ~ N(0, 3^2); a fraction of (part, row)
+    entries saw no key (lse -inf), and the last row saw none in any part."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    out = _randn_fp16(gen, (parts, rows, head_dim))
+    lse = torch.randn((parts, rows), generator=gen, dtype=torch.float32) * 3.0
+    empty = torch.rand((parts, rows), generator=gen) < empty_frac
+    lse[empty] = float("-inf")
+    if rows:
+        lse[:, -1] = float("-inf")
+    return out, lse

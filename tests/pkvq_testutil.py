@@ -26,7 +26,8 @@ def oracle_cache(case: synth.Case) -> oracle.Cache:
     s = case.spec
     c = oracle.Cache(s.kv_dtype, case.num_blocks, s.block_size, s.num_kv_heads, s.head_dim,
                      None if case.k_scale is None else case.k_scale.numpy(),
-                     None if case.v_scale is None else case.v_scale.numpy())
+                     None if case.v_scale is None else case.v_scale.numpy(),
+                     scale_per_layer=s.scale_per_layer)
     c.write(bits16(case.k), bits16(case.v), case.slot_mapping.numpy())
     return c
 
@@ -38,8 +39,9 @@ def gpu_cache(case: synth.Case, poison: bool = True, write: bool = True) -> pk.P
     s = case.spec
     cache = pk.PagedKVCache.allocate(s.kv_dtype, case.num_blocks, s.block_size,
                                      s.num_kv_heads, s.head_dim, k_scale=case.k_scale,
-                                     v_scale=case.v_scale)
+                                     v_scale=case.v_scale, scale_per_layer=s.scale_per_layer)
     if poison:
+        # 0x7F: a NaN code of E4M3 and E5M2; 0x7F7F: an fp16 NaN
         cache.k_cache.fill_(NAN_E4M3)
         cache.v_cache.fill_(NAN_E4M3)
         if cache.k_scale_tok is not None:
@@ -66,6 +68,7 @@ def assert_codes_equal(cache: pk.PagedKVCache, oc: oracle.Cache, case: synth.Cas
     for name in ("k_cache", "v_cache"):
         g = getattr(cache, name).cpu().numpy()
         o = getattr(oc, name)
+        assert g.shape == o.shape, (g.shape, o.shape)
         gw = g.transpose(0, 2, 1, 3)[m]
         ow = o.transpose(0, 2, 1, 3)[m]
         bad = np.nonzero(gw != ow)
@@ -78,19 +81,25 @@ def assert_codes_equal(cache: pk.PagedKVCache, oc: oracle.Cache, case: synth.Cas
             assert np.array_equal(g, o), f"{name} differs"
 
 
-def run_gpu(case: synth.Case, cache: pk.PagedKVCache, want_lse: bool = True):
+def run_gpu(case: synth.Case, cache: pk.PagedKVCache, want_lse: bool = True,
+            block_table=None, context_lens=None, query_pos=None):
+    """The case through the C ABI; block_table / context_lens / query_pos
+    (decode) replace the case's own, e.g. for one rank's share of the keys."""
     s = case.spec
     dev = "cuda"
-    bt = case.block_table.to(dev)
-    ctx = case.context_lens.to(dev)
+    bt = (case.block_table if block_table is None else block_table).to(dev)
+    ctx = (case.context_lens if context_lens is None else context_lens).to(dev)
     if s.kind == "decode":
         B = len(s.context_lens)
         ql = s.q_lens[0]
         q = case.q.view(B, ql, s.num_q_heads, s.head_dim).to(dev)
         lse = torch.empty((B, ql, s.num_q_heads), dtype=torch.float32, device=dev) \
             if want_lse else None
-        out = pk.paged_attn_decode(cache, q, bt, ctx, max(s.context_lens + [0]),
-                                   case.softmax_scale, lse=lse)
+        qp = None if query_pos is None else query_pos.view(B, ql).to(dev)
+        lens = s.context_lens if context_lens is None else context_lens.tolist()
+        out = pk.paged_attn_decode(cache, q, bt, ctx, max(list(lens) + [0]),
+                                   case.softmax_scale, lse=lse, sliding_window=s.window,
+                                   query_pos=qp)
         out = out.view(-1, s.num_q_heads, s.head_dim)
         lse = None if lse is None else lse.view(-1, s.num_q_heads)
     else:
@@ -98,7 +107,8 @@ def run_gpu(case: synth.Case, cache: pk.PagedKVCache, want_lse: bool = True):
         lse = torch.empty((q.shape[0], s.num_q_heads), dtype=torch.float32, device=dev) \
             if want_lse else None
         out = pk.paged_attn_prefill(cache, q, case.cu_seqlens_q.to(dev), bt, ctx,
-                                    max(s.q_lens + [0]), case.softmax_scale, lse=lse)
+                                    max(s.q_lens + [0]), case.softmax_scale, lse=lse,
+                                    sliding_window=s.window)
     torch.cuda.synchronize()
     return out.cpu(), (None if lse is None else lse.cpu())
 
@@ -106,7 +116,7 @@ def run_gpu(case: synth.Case, cache: pk.PagedKVCache, want_lse: bool = True):
 def run_oracle(case: synth.Case, oc: oracle.Cache, rows=None):
     return oracle.paged_attention(oc, bits16(case.q), case.cu_seqlens_q.numpy(),
                                   case.context_lens.numpy(), case.block_table.numpy(),
-                                  case.softmax_scale, rows=rows)[:2]
+                                  case.softmax_scale, rows=rows, window=case.spec.window)[:2]
 
 
 def abs_value_oracle(case: synth.Case, oc: oracle.Cache, rows=None) -> np.ndarray:

@@ -165,7 +165,8 @@ def test_verify_rows_take_the_tensor_core_plan(lib, monkeypatch):
     monkeypatch.delenv("PKVQ_DECODE_CTAS_PER_SM", raising=False)
     sms, hkv, rows, batch = 148, 4, 40, 6
     C = max(batch, sms // hkv)
-    assert _ws(lib, batch, 5, 32, hkv, 524288) == hkv * C * rows * (128 + 2) * 4
+    counters = 16 * sms * 4   # the leading counter area (already a multiple of 256)
+    assert _ws(lib, batch, 5, 32, hkv, 524288) == counters + hkv * C * rows * (128 + 2) * 4
 
 
 def test_row_counts_past_one_tile_use_row_groups(lib, monkeypatch):
@@ -176,10 +177,68 @@ def test_row_counts_past_one_tile_use_row_groups(lib, monkeypatch):
     groups = 256 // 16
     units = hkv * groups
     C = max(batch, 2 * sms // units)
-    assert _ws(lib, batch, 16, 32, hkv, 65536) == units * C * 16 * (128 + 2) * 4
+    assert _ws(lib, batch, 16, 32, hkv, 65536) == 16 * sms * 4 + units * C * 16 * (128 + 2) * 4
 
 
 def test_one_slot_per_sequence_needs_no_workspace(lib, monkeypatch):
     # more sequences than the GPU has slots for: every sequence is one split
     monkeypatch.setenv("PKVQ_DECODE_CTAS_PER_SM", "1")
     assert _ws(lib, 4096, 1, 32, 4, 32768) == 0
+
+
+# ---- the entry points added for the next rows (host-side checks only) ----
+
+def test_decode_ex_and_prefill_ex_option_checks(lib):
+    c = _cache()
+    P = ctypes.c_void_p
+    bad = pk.AttnOpts(-1, None)
+    rc = lib.pkvq_paged_attn_decode_ex(ctypes.byref(c), P(0x10000), P(0x20000), None,
+                                       P(0x30000), 64, P(0x40000), 2, 1, 8, 1024,
+                                       ctypes.c_float(0.088), ctypes.byref(bad), None, 0, None)
+    assert rc == INVALID
+    qp = pk.AttnOpts(0, 0x50000)
+    rc = lib.pkvq_paged_attn_prefill_ex(ctypes.byref(c), P(0x10000), P(0x20000), None,
+                                        P(0x30000), P(0x40000), 64, P(0x50000), 1, 16, 8,
+                                        ctypes.c_float(0.088), ctypes.byref(qp), None, 0, None)
+    assert rc == UNSUPPORTED        # query positions are a decode option
+    # a zeroed options struct is the plain call: batch 0 is still a no-op
+    z = pk.AttnOpts(0, None)
+    rc = lib.pkvq_paged_attn_decode_ex(ctypes.byref(c), P(0x10000), P(0x20000), None,
+                                       P(0x30000), 64, P(0x40000), 0, 1, 8, 1024,
+                                       ctypes.c_float(0.088), ctypes.byref(z), None, 0, None)
+    assert rc == 0
+
+
+def test_new_formats_are_accepted_and_checked(lib):
+    # E5M2 needs its fp32 scales like E4M3; FP16 needs none
+    assert lib.pkvq_kv_write_quant(ctypes.byref(_cache(dtype=2, k_scale=None)),
+                                   ctypes.c_void_p(16), ctypes.c_void_p(16),
+                                   ctypes.c_void_p(16), 1, None) == INVALID
+    assert lib.pkvq_decode_workspace_bytes(2, 1, 8, 4096,
+                                           ctypes.byref(_cache(dtype=3, k_scale=None,
+                                                               v_scale=None))) > 0
+    assert lib.pkvq_decode_workspace_bytes(2, 1, 8, 4096, ctypes.byref(_cache(dtype=2))) > 0
+
+
+def test_merge_argument_checks(lib):
+    P = ctypes.c_void_p
+    m = lambda **kw: lib.pkvq_merge_attn_states(
+        P(kw.get("po", 0x1000)), P(kw.get("pl", 0x2000)), kw.get("R", 2), kw.get("n", 4),
+        kw.get("D", 128), P(kw.get("out", 0x3000)), None, None)
+    assert m(D=64) == UNSUPPORTED
+    assert m(R=0) == INVALID and m(R=65) == INVALID and m(n=-1) == INVALID
+    assert m(po=None) == INVALID and m(out=None) == INVALID
+    assert m(out=0x3008) == MISALIGNED
+    assert m(n=0, po=None) == 0     # no rows: no-op
+
+
+def test_copy_blocks_argument_checks(lib):
+    P = ctypes.c_void_p
+    a, b = _cache(), _cache(num_blocks=9)
+    assert lib.pkvq_kv_copy_blocks(ctypes.byref(a), ctypes.byref(b), P(0x5000), -1, None) == INVALID
+    assert lib.pkvq_kv_copy_blocks(ctypes.byref(a), ctypes.byref(b), None, 3, None) == INVALID
+    assert lib.pkvq_kv_copy_blocks(ctypes.byref(a), ctypes.byref(b), None, 0, None) == 0
+    for kw in (dict(block_size=32), dict(num_kv_heads=4), dict(dtype=1, k_scale_tok=0x7000,
+                                                               v_scale_tok=0x8000)):
+        assert lib.pkvq_kv_copy_blocks(ctypes.byref(a), ctypes.byref(_cache(**kw)), P(0x5000),
+                                       1, None) == INVALID

@@ -162,3 +162,118 @@ def test_decode_workspace_too_small_is_rejected():
         pk.paged_attn_decode(cache, q, case.block_table.cuda(), case.context_lens.cuda(), 8192,
                              case.softmax_scale, workspace=ws)
     assert e.value.status == 4
+
+
+# ------------------------------------------------ E5M2, FP16, layer scale --
+
+FORMAT_CASES = [
+    # dtype, Hq, Hkv, ctx list, q_len, bs, per-layer scale
+    (synth.FP8_E5M2, 32, 4, [777, 16, 1, 2049], 1, 16, False),   # mma.sync, 8 rows
+    (synth.FP8_E5M2, 16, 1, [513], 1, 32, True),                  # 16 rows, layer scale
+    (synth.FP8_E5M2, 32, 4, [999, 17], 5, 64, False),             # tcgen05, 40 rows
+    (synth.FP16, 32, 4, [777, 16, 1, 2049], 1, 16, False),
+    (synth.FP16, 8, 4, [300, 129], 1, 64, False),
+    (synth.FP16, 16, 2, [1000, 333], 3, 32, False),               # tcgen05, 24 rows
+    (synth.FP16, 32, 4, [4000, 5, 900], 5, 16, False),            # tcgen05, 40 rows
+    (synth.FP16, 32, 4, [20000, 3], 2, 16, False),                # 16 rows, many splits
+    (synth.FP8_E4M3, 32, 4, [5000, 77], 1, 16, True),             # E4M3, layer scale
+    (synth.FP8_E4M3, 32, 4, [3000, 300], 5, 32, True),            # tcgen05, layer scale
+]
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,ctx,ql,bs,per_layer", FORMAT_CASES)
+def test_decode_new_formats_match_oracle(dtype, Hq, Hkv, ctx, ql, bs, per_layer):
+    case = _case(dtype, Hq, Hkv, ctx, ql, bs, seed=22, outlier_frac=0.01,
+                 scale_per_layer=per_layer)
+    cache = gpu_cache(case)
+    oc = oracle_cache(case)
+    assert_codes_equal(cache, oc, case)
+    out, lse = run_gpu(case, cache)
+    ref, ref_lse = run_oracle(case, oc)
+    assert_matches_oracle(case, oc, out, lse, ref, ref_lse,
+                          what=f"decode fmt {dtype} {Hq}/{Hkv} {ctx} q{ql} bs{bs} L{per_layer}")
+    assert pk.device_status() == 0
+
+
+# ---------------------------------------------------------- sliding window --
+
+WINDOW_CASES = [
+    # dtype, Hq, Hkv, ctx list, q_len, bs, window
+    (FP8, 8, 2, [3000, 100, 17, 0], 1, 16, 500),       # mma.sync; windows past and inside
+    (FP8, 32, 4, [16384, 700], 1, 16, 4096),           # many splits inside the window
+    (INT8, 16, 4, [2000, 65], 3, 32, 129),             # 12 rows, window of one row + 1
+    (INT8, 32, 4, [5000, 64, 3], 5, 16, 1000),         # tcgen05, 40 rows
+    (synth.FP16, 16, 2, [3000], 4, 64, 200),           # tcgen05, FP16
+    (synth.FP8_E5M2, 8, 2, [999], 2, 16, 1),           # window 1: each row its own key
+]
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,ctx,ql,bs,window", WINDOW_CASES)
+def test_decode_sliding_window_matches_oracle(dtype, Hq, Hkv, ctx, ql, bs, window):
+    case = _case(dtype, Hq, Hkv, ctx, ql, bs, seed=23, window=window)
+    case.spec.context_lens = list(ctx)
+    cache = gpu_cache(case)
+    oc = oracle_cache(case)
+    out, lse = run_gpu(case, cache)
+    ref, ref_lse = run_oracle(case, oc)
+    assert_matches_oracle(case, oc, out, lse, ref, ref_lse,
+                          what=f"decode window {window} {dtype} {ctx} q{ql} bs{bs}")
+    assert pk.device_status() == 0
+
+
+# ---------------------------------- sequence-sharded decode (query positions) --
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("dtype,Hq,Hkv,ctx,ql,bs", [
+    (FP8, 32, 4, [32768, 5000, 16, 1], 1, 16),          # mma.sync path on every rank
+    (INT8, 32, 4, [20000, 3000, 7], 5, 16),             # tcgen05 path, verify rows
+    (synth.FP16, 16, 2, [4096, 100], 2, 32),
+])
+def test_sharded_decode_merged_matches_oracle(world, dtype, Hq, Hkv, ctx, ql, bs):
+    # one GPU plays every rank in turn: each decodes its share of every
+    # sequence's blocks at its queries' local positions; the merge kernel
+    # combines the per-rank (out, lse) pairs
+    case = _case(dtype, Hq, Hkv, ctx, ql, bs, seed=24)
+    cache = gpu_cache(case)
+    oc = oracle_cache(case)
+    outs, lses = [], []
+    for r in range(world):
+        sh = synth.dcp_shard(case, world, r)
+        o, l = run_gpu(case, cache, block_table=sh.block_table, context_lens=sh.context_lens,
+                       query_pos=sh.query_pos)
+        outs.append(o)
+        lses.append(l)
+    out, lse = pk.merge_attn_states(torch.stack(outs).cuda(), torch.stack(lses).cuda())
+    torch.cuda.synchronize()
+    ref, ref_lse = run_oracle(case, oc)
+    assert_matches_oracle(case, oc, out.cpu(), lse.cpu(), ref, ref_lse,
+                          what=f"sharded x{world} {dtype} {ctx} q{ql}")
+    assert pk.device_status() == 0
+
+
+def test_decode_workspace_reused_across_shapes():
+    # One zero-filled workspace serves calls of different shapes in turn: the
+    # arrival counters sit in a leading area that no call's partials touch,
+    # and each call returns them to zero.
+    ws = torch.zeros(48 << 20, dtype=torch.uint8, device="cuda")
+    specs = [
+        (FP8, 32, 4, [16384, 300, 5000], 1, 16),    # mma.sync, merged by its last CTAs
+        (INT8, 32, 4, [9000, 17], 5, 16),           # tcgen05 (keys on M), merge kernel
+        (FP8, 16, 2, [20000, 4000], 1, 32),         # mma.sync again, other partial sizes
+        (INT8, 16, 4, [3000, 12000, 64], 1, 16),
+    ]
+    for dtype, Hq, Hkv, ctx, ql, bs in specs:
+        case = _case(dtype, Hq, Hkv, ctx, ql, bs, seed=25)
+        cache = gpu_cache(case)
+        B = len(ctx)
+        q = case.q.view(B, ql, Hq, 128).cuda()
+        bt, cl = case.block_table.cuda(), case.context_lens.cuda()
+        assert pk.decode_workspace_bytes(cache, B, ql, Hq, max(ctx)) <= ws.numel()
+        shared = pk.paged_attn_decode(cache, q, bt, cl, max(ctx), case.softmax_scale,
+                                      workspace=ws)
+        fresh = pk.paged_attn_decode(cache, q, bt, cl, max(ctx), case.softmax_scale)
+        torch.cuda.synchronize()
+        assert torch.equal(shared, fresh)
+    # the counter area is back to zero
+    assert int(ws[: 16 * 148 * 4].view(torch.int32).abs().max()) == 0
+    assert pk.device_status() == 0

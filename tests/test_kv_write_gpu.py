@@ -106,3 +106,54 @@ def test_zero_tokens_is_a_noop():
 
 def test_device_status_clean_after_writes():
     assert pk.device_status(clear=True) == 0
+
+
+# ------------------------------------------------ E5M2, FP16, layer scale --
+
+@pytest.mark.parametrize("scale", [1.0, 0.125, 0.0123, 90.0 / 57344, 3.0e-5, 0.0])
+def test_e5m2_every_fp16_pattern(scale):
+    k = _all_fp16_rows(finite_only=False)                 # includes inf and NaN patterns
+    v = torch.flip(k, dims=[0]).contiguous()
+    T = k.shape[0]
+    slots = torch.randperm(T, generator=torch.Generator().manual_seed(5)).to(torch.int32)
+    cache, oc = _write_both(synth.FP8_E5M2, k, v, slots, T // 16, 16, 1,
+                            k_scale=[scale], v_scale=[scale * 2])
+    for name in ("k_cache", "v_cache"):
+        g = getattr(cache, name).cpu().numpy()
+        o = getattr(oc, name)
+        assert np.array_equal(g, o), f"{name}: {(g != o).sum()} codes differ"
+
+
+def test_fp16_cache_holds_every_pattern_bit_for_bit():
+    k = _all_fp16_rows(finite_only=False)
+    v = torch.flip(k, dims=[0]).contiguous()
+    T = k.shape[0]
+    slots = torch.randperm(T, generator=torch.Generator().manual_seed(6)).to(torch.int32)
+    cache, oc = _write_both(synth.FP16, k, v, slots, T // 32, 32, 1)
+    for name in ("k_cache", "v_cache"):
+        assert np.array_equal(getattr(cache, name).cpu().numpy(), getattr(oc, name)), name
+
+
+@pytest.mark.parametrize("dtype", [synth.FP8_E4M3, synth.FP8_E5M2])
+def test_per_layer_scale_write(dtype):
+    spec = synth.CaseSpec("decode", dtype, 8, 4, [300, 7], [1, 1], outlier_frac=0.02,
+                          scale_per_layer=True, seed=8)
+    case = synth.make_case(spec)
+    assert case.k_scale.shape == (1,)
+    cache = gpu_cache(case)
+    oc = oracle_cache(case)
+    assert_codes_equal(cache, oc, case)
+
+
+@pytest.mark.parametrize("dtype", [synth.FP8_E5M2, synth.FP16])
+@pytest.mark.parametrize("bs", [16, 32, 64])
+def test_new_formats_ragged_and_skipped(dtype, bs):
+    spec = synth.CaseSpec("decode", dtype, 8, 4, [37, 1, 300], [1, 1, 1], block_size=bs,
+                          outlier_frac=0.02, seed=9)
+    case = synth.make_case(spec)
+    case.slot_mapping[5] = -1
+    cache = gpu_cache(case)
+    oc = oracle_cache(case)
+    keep = case.slot_mapping >= 0
+    case.slot_mapping = case.slot_mapping[keep]
+    assert_codes_equal(cache, oc, case)

@@ -81,3 +81,31 @@ def test_prefill_matches_decode_on_the_last_token():
     torch.cuda.synchronize()
     d = (out_d.view(16, 128).cpu().float() - out_p[-1].float()).abs().max().item()
     assert d <= 2e-3
+
+
+# ------------------------------------- E5M2, FP16, layer scale, window --
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,ctx,ql,bs,per_layer,window", [
+    (synth.FP8_E5M2, 32, 4, [200, 1000], [200, 37], 16, False, 0),
+    (synth.FP8_E5M2, 8, 2, [700], [300], 64, True, 0),
+    (synth.FP16, 8, 1, [300], [300], 16, False, 0),
+    (synth.FP16, 32, 4, [1100, 70], [300, 70], 32, False, 0),
+    (synth.FP16, 12, 2, [260], [130], 64, False, 0),
+    (FP8, 32, 4, [2500], [1024], 16, True, 0),
+    (FP8, 8, 2, [1000], [1000], 16, False, 100),          # window: loop starts late
+    (INT8, 32, 4, [3000], [700], 16, False, 257),
+    (synth.FP16, 16, 2, [600, 90], [600, 90], 64, False, 64),
+    (synth.FP8_E5M2, 8, 8, [129, 64], [129, 1], 32, False, 1),
+    (FP8, 32, 4, [5000], [300], 16, False, 4000),         # window longer than the chunk
+])
+def test_prefill_new_formats_and_window(dtype, Hq, Hkv, ctx, ql, bs, per_layer, window):
+    spec = synth.CaseSpec("prefill", dtype, Hq, Hkv, list(ctx), list(ql), block_size=bs,
+                          seed=32, outlier_frac=0.01, scale_per_layer=per_layer, window=window)
+    case = synth.make_case(spec)
+    cache = gpu_cache(case)
+    oc = oracle_cache(case)
+    out, lse = run_gpu(case, cache)
+    ref, ref_lse = run_oracle(case, oc)
+    assert_matches_oracle(case, oc, out, lse, ref, ref_lse,
+                          what=f"prefill {dtype} {ctx} {ql} bs{bs} L{per_layer} w{window}")
+    assert pk.device_status() == 0
