@@ -14,6 +14,7 @@ import glob
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -52,12 +53,15 @@ def build(force: bool = False, bounds_check: bool = False, verbose: bool = False
         flags.append("-DPKVQ_BOUNDS_CHECK")
     if verbose:
         flags += ["-Xptxas", "-v"]
-    objs = []
-    for src in _sources():
+    def compile_one(src):
         obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
-        cmd = [NVCC] + flags + ["-c", src, "-o", obj]
-        subprocess.run(cmd, check=True)
-        objs.append(obj)
+        subprocess.run([NVCC] + flags + ["-c", src, "-o", obj], check=True)
+        return obj
+
+    # translation units compile independently (the tensor-core ones take
+    # about a minute each)
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        objs = list(ex.map(compile_one, _sources()))
     tmp = out + f".tmp{os.getpid()}"
     subprocess.run([NVCC] + ARCH + ["-shared", "-o", tmp] + objs, check=True)
     os.replace(tmp, out)

@@ -298,6 +298,8 @@ pkvq_status pkvq_paged_attn_decode_ex(const pkvq_cache *cache, const void *q, vo
     if (st != PKVQ_OK)
         return st;
     DecodeParams p{};
+    p.k_cache = static_cast<const uint8_t *>(cache->k_cache);
+    p.v_cache = static_cast<const uint8_t *>(cache->v_cache);
     const bool head_scale = kv_has_head_scale(cache->dtype);
     p.k_scale = head_scale ? cache->k_scale : nullptr;
     p.v_scale = head_scale ? cache->v_scale : nullptr;
@@ -392,6 +394,8 @@ pkvq_status pkvq_paged_attn_prefill_ex(const pkvq_cache *cache, const void *q, v
     if (st != PKVQ_OK)
         return st;
     PrefillParams p{};
+    p.k_cache = static_cast<const uint8_t *>(cache->k_cache);
+    p.v_cache = static_cast<const uint8_t *>(cache->v_cache);
     const bool head_scale = kv_has_head_scale(cache->dtype);
     p.k_scale = head_scale ? cache->k_scale : nullptr;
     p.v_scale = head_scale ? cache->v_scale : nullptr;

@@ -997,7 +997,7 @@ cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_
     cudaError_t e;
     const bool one = plan.nt == 1;
     if (plan.tn)
-        e = launch_decode_tn(p, kv_dtype, kmap, vmap, stream);
+        e = launch_decode_tn(p, kv_dtype, stream);
     else if (plan.tc)
         e = launch_decode_tc(p, kv_dtype, kmap, vmap, stream);
     else if (kv_dtype == kKvFp8)

@@ -38,6 +38,7 @@ struct KvWriteParams {
 cudaError_t launch_kv_write_quant(const KvWriteParams &p, int kv_dtype, cudaStream_t stream);
 
 struct DecodeParams {
+    const uint8_t *k_cache, *v_cache;            // [blocks][Hkv][block_size][row bytes]
     const float *k_scale, *v_scale;              // FP8 formats: per KV head (or layer)
     int scale_stride;                            // 1: per KV head; 0: one per layer
     const uint16_t *k_scale_tok, *v_scale_tok;   // INT8: per (block, head, token)
@@ -89,14 +90,14 @@ bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv
 // rows on the MMA's M (65..128 rows) or keys on M (17..64 rows).
 cudaError_t launch_decode_tc(const DecodeParams &p, int kv_dtype, const CUtensorMap &kmap,
                              const CUtensorMap &vmap, cudaStream_t stream);
-cudaError_t launch_decode_tn(const DecodeParams &p, int kv_dtype, const CUtensorMap &kmap,
-                             const CUtensorMap &vmap, cudaStream_t stream);
+cudaError_t launch_decode_tn(const DecodeParams &p, int kv_dtype, cudaStream_t stream);
 
 cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_dtype,
                           const CUtensorMap &kmap, const CUtensorMap &vmap,
                           cudaStream_t stream);
 
 struct PrefillParams {
+    const uint8_t *k_cache, *v_cache;            // [blocks][Hkv][block_size][row bytes]
     const float *k_scale, *v_scale;
     int scale_stride;                            // 1: per KV head; 0: one per layer
     const uint16_t *k_scale_tok, *v_scale_tok;

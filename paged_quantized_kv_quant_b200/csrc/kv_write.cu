@@ -7,11 +7,12 @@
 //
 // One (token, KV head) row of head_dim = 128 fp16 values is handled by a
 // group of 16 threads; each thread owns 8 consecutive elements, i.e. one
-// 16-byte load of K and one of V.  A group takes kRowsPerGroup rows and
-// issues all of their loads before converting any, so that every thread has
-// kRowsPerGroup x 32 bytes in flight.  The kernel is a single bandwidth-bound
-// pass: 512 bytes read and 256 bytes of codes (512 for FP16, +4 bytes of
-// INT8 scales) written per row.
+// 16-byte load of K and one of V.  (A group can take kRowsPerGroup rows and
+// issue all of their loads before converting any; more than one row per group
+// measured slower: the IEEE divisions of the FP8 formats then serialize per
+// thread, and the one-token writes of a decode step lose most of their
+// parallelism.)  The kernel is a single pass: 512 bytes read and 256 bytes
+// of codes (512 for FP16, +4 bytes of INT8 scales) written per row.
 #include "common.cuh"
 #include "internal.h"
 
@@ -25,7 +26,7 @@ constexpr int kThreadsPerRow = 16;
 constexpr int kElemsPerThread = 8;
 constexpr int kBlockThreads = 256;
 constexpr int kGroupsPerBlock = kBlockThreads / kThreadsPerRow;
-constexpr int kRowsPerGroup = 4;
+constexpr int kRowsPerGroup = 1;
 constexpr int kRowsPerBlock = kGroupsPerBlock * kRowsPerGroup;
 
 // fp32 quotient -> E4M3 / E5M2 with round-to-nearest-even and saturation to

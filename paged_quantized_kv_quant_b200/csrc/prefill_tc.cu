@@ -43,6 +43,7 @@
 // window start.
 #include "common.cuh"
 #include "internal.h"
+#include "kv_stage.cuh"
 #include "tc.cuh"
 
 #include <climits>
@@ -55,6 +56,9 @@ constexpr int kThreads = 384;
 constexpr int kKT = 64;              // keys per tile
 constexpr int kCodeStages = 3;
 constexpr int kKVBufs = 4;           // dequantised K/V tiles in flight
+// L2 prefetch distance in tiles: with 16-token blocks the farthest prefetched
+// block stays within 60 entries of the block-table window's base
+constexpr int kPrefetchTiles = 6;
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
 
@@ -165,6 +169,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                   const __grid_constant__ CUtensorMap vmap, const PrefillParams p)
 {
     constexpr int kBPT = kKT / BS;   // cache blocks per key tile
+    static_assert((kPrefetchTiles + 1) * kBPT <= 32, "prefetches stay in the table window");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -196,13 +201,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     if (tid == 0) {
         mbar_init(bars.q_full, 8);
         for (int s = 0; s < kCodeStages; ++s) {
-            mbar_init(&bars.code_full[s], 1);
+            mbar_init(&bars.code_full[s], 32);   // one cp.async arrival per producer lane
             mbar_init(&bars.code_empty[s], kDequantWarps);
         }
         for (int i = 0; i < kKVBufs; ++i) {
             mbar_init(&bars.kv_full[i], kDequantWarps);
             mbar_init(&bars.kv_empty[i], 1);
-            mbar_init(&bars.kv_tma[i], 1);
+            mbar_init(&bars.kv_tma[i], 32);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars.s_full[i], 1);
@@ -222,104 +227,49 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     const uint32_t tmem = *taddr_smem;
 
     if (warp == kWarpTma) {
-        // ------------------------------------------------ TMA producer --
-        if (lane == 0) {
-            prefetch_tmap(&kmap);
-            prefetch_tmap(&vmap);
-        }
-        const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq + blk_base;
+        // ---------------------------------------------- copy producer --
+        // 16-byte cp.async copies by all 32 lanes; each lane arrives on the
+        // tile's barrier once its own copies have landed.  The tiles up to
+        // kPrefetchTiles past the one being loaded are first fetched into L2.
+        const CacheView cv{p.k_cache, p.v_cache, p.k_scale_tok, p.v_scale_tok, p.num_kv_heads,
+                           p.num_blocks, p.status};
+        BlockWindow w;
         // every index stays inside the table row, even for a context longer
         // than the row can address (a caller error: those keys read block 0)
-        const int nblk_used =
-            min(min(nblk_seq - blk_base, ntiles * kBPT), p.max_blocks_per_seq - blk_base);
-        int win0 = lane < nblk_used ? __ldg(bt + lane) : 0;
-        int win1 = 32 + lane < nblk_used ? __ldg(bt + 32 + lane) : 0;
-        int wbase = 0;
-        int issued = 0;
+        w.init(p.block_table + (size_t)b * p.max_blocks_per_seq + blk_base,
+               min(min(nblk_seq - blk_base, ntiles * kBPT), p.max_blocks_per_seq - blk_base),
+               lane);
         // FP16: each tile goes straight into K/V buffer j % kKVBufs
         constexpr int kRing = KVT == kKvFp16 ? kKVBufs : kCodeStages;
+        int pf_next = kRing;
         for (int j = 0; j < ntiles; ++j) {
+            for (; pf_next < ntiles && pf_next <= j + kPrefetchTiles; ++pf_next)
+                prefetch_blocks<BS, KVT>(cv, h, w, pf_next * kBPT,
+                                         min(kBPT, nblk_seq - blk_base - pf_next * kBPT), lane);
             const int s = j % kRing;
             uint64_t *empty = KVT == kKvFp16 ? bars.kv_empty : bars.code_empty;
             if (j >= kRing && !warp_wait(&empty[s], ((j - kRing) / kRing) & 1, p.status))
                 break;
-            issued = j + 1;
             const int blk0 = j * kBPT;   // from blk_base
             const int nb = min(kBPT, nblk_seq - blk_base - blk0);
-            int ids[kBPT];
-#pragma unroll
-            for (int i = 0; i < kBPT; ++i) {
-                const int bi = blk0 + i;
-                const int a = __shfl_sync(0xffffffffu, win0, bi & 31);
-                const int c = __shfl_sync(0xffffffffu, win1, bi & 31);
-                ids[i] = (bi - wbase) < 32 ? a : c;
-            }
-            if (KVT == kKvFp16 && lane == 0) {
-                mbar_arrive_expect_tx(&bars.kv_tma[s], (uint32_t)nb * BS * 256 * 2);
-                uint8_t *kv = smem + kOffKV + s * kKVBuf;
-#pragma unroll
-                for (int i = 0; i < kBPT; ++i) {
-                    if (i >= nb)
-                        break;
-                    int phys = ids[i];
-#ifdef PKVQ_BOUNDS_CHECK
-                    if (phys < 0 || phys >= p.num_blocks) {
-                        atomicOr(p.status, kStatusBadBlock);
-                        phys = 0;
-                    }
-#endif
-                    const int y = (phys * p.num_kv_heads + h) * BS;
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        tma_tile_2d_g2s(kv + half * 8192 + i * BS * 128, &kmap, 128 * half, y,
-                                        &bars.kv_tma[s]);
-                        tma_tile_2d_g2s(kv + 16384 + half * 8192 + i * BS * 128, &vmap,
-                                        128 * half, y, &bars.kv_tma[s]);
-                    }
+            if constexpr (KVT == kKvFp16) {
+                const uint32_t kv = sbase + kOffKV + s * kKVBuf;
+                copy_fp16_rows<BS>(kv, kv + 16384, 8192, cv, h, w, blk0, nb, kKT, lane);
+                cp_async_mbar_arrive(&bars.kv_tma[s]);
+            } else {
+                const uint32_t dst = sbase + kOffCodes + s * kCodeStage;
+                copy_code_rows<BS>(dst, dst + 8192, cv, h, w, blk0, nb, kKT, lane);
+                if constexpr (KVT == kKvInt8) {
+                    const uint32_t sd = sbase + kOffScl + s * 256;
+                    copy_int8_scales<BS>(sd, sd + 128, cv, h, w, blk0, nb, lane);
                 }
-            } else if (lane == 0) {
-                uint32_t tx = (uint32_t)nb * BS * 128 * 2;
-                if constexpr (KVT == kKvInt8)
-                    tx += (uint32_t)nb * BS * 2 * 2;
-                mbar_arrive_expect_tx(&bars.code_full[s], tx);
-                uint8_t *dst = smem + kOffCodes + s * kCodeStage;
-                uint16_t *sd = reinterpret_cast<uint16_t *>(smem + kOffScl + s * 256);
-#pragma unroll
-                for (int i = 0; i < kBPT; ++i) {
-                    if (i >= nb)
-                        break;
-                    int phys = ids[i];
-#ifdef PKVQ_BOUNDS_CHECK
-                    if (phys < 0 || phys >= p.num_blocks) {
-                        atomicOr(p.status, kStatusBadBlock);
-                        phys = 0;
-                    }
-#endif
-                    const int y = (phys * p.num_kv_heads + h) * BS;
-                    tma_tile_2d_g2s(dst + i * BS * 128, &kmap, 0, y, &bars.code_full[s]);
-                    tma_tile_2d_g2s(dst + 8192 + i * BS * 128, &vmap, 0, y, &bars.code_full[s]);
-                    if constexpr (KVT == kKvInt8) {
-                        tma_bulk_g2s(sd + i * BS, p.k_scale_tok + (size_t)y, BS * 2,
-                                     &bars.code_full[s]);
-                        tma_bulk_g2s(sd + 64 + i * BS, p.v_scale_tok + (size_t)y, BS * 2,
-                                     &bars.code_full[s]);
-                    }
-                }
+                cp_async_mbar_arrive(&bars.code_full[s]);
             }
-            if (blk0 + kBPT >= wbase + 32) {
-                wbase += 32;
-                win0 = win1;
-                win1 = wbase + 32 + lane < nblk_used ? __ldg(bt + wbase + 32 + lane) : 0;
-            }
+            if (j + 1 < ntiles)
+                w.slide(blk0 + kBPT, lane);
         }
-        // Copies this CTA issued must land before it exits: wait (bounded) for
-        // the most recent round of every stage (already complete when the
-        // consumers kept up).
-        if (lane == 0) {
-            uint64_t *full = KVT == kKvFp16 ? bars.kv_tma : bars.code_full;
-            for (int j = max(0, issued - kRing); j < issued; ++j)
-                mbar_wait(&full[j % kRing], (j / kRing) & 1, nullptr);
-        }
+        // copies this warp issued land before it exits
+        cp_async_wait_all();
     } else if (warp == kWarpMma) {
         // --------------------------------------------------- MMA issuer --
         // Serves whichever query tile has its P ready (no head-of-line

@@ -36,6 +36,9 @@ CASES = [
     # more than 16 rows per KV head: the tcgen05 kernel, every block size
     (FP8, 16, 2, [1000, 333], 3, 32),       # 24 rows
     (INT8, 8, 1, [2000, 77], 4, 64),        # 32 rows
+    (INT8, 16, 2, [3000, 129], 6, 16),      # 48 rows
+    (FP8, 32, 4, [2500, 1], 7, 32),         # 56 rows
+    (INT8, 16, 2, [1300, 700], 8, 16),      # 64 rows: the widest keys-on-M tile
     (FP8, 16, 2, [900], 16, 16),            # 128 rows: one full tile
     (FP8, 32, 2, [500], 16, 16),            # 256 rows: past the tile, mma.sync row groups
 ]
