@@ -33,13 +33,20 @@ def _write_both(dtype, k, v, slots, num_blocks, bs, Hkv, k_scale=None, v_scale=N
     return cache, oc
 
 
-@pytest.mark.parametrize("scale", [1.0, 0.125, 0.0123, 4.4 / 448, 3.0e-5, 0.0])
-def test_fp8_every_fp16_pattern(scale):
+# Power-of-two scales put every fp16 value exactly on its quotient, so the
+# E4M3 / E5M2 rounding midpoints among fp16 values are hit exactly (ties to
+# even); 1 +- 2^-22 moves them a fraction of an fp32 ulp off the midpoints,
+# where a product with the rounded reciprocal can round the other way; tiny
+# and huge scales take the quotient to both ends of the fp32 range.
+@pytest.mark.parametrize("dtype", [synth.FP8_E4M3, synth.FP8_E5M2])
+@pytest.mark.parametrize("scale", [1.0, 0.125, 0.0123, 4.4 / 448, 3.0e-5, 0.0,
+                                   1.0 + 2.0 ** -22, 1.0 - 2.0 ** -22, 1.0e-38, 3.0e37])
+def test_fp8_every_fp16_pattern(dtype, scale):
     k = _all_fp16_rows(finite_only=False)                 # includes inf and NaN patterns
     v = torch.flip(k, dims=[0]).contiguous()
     T = k.shape[0]
     slots = torch.randperm(T, generator=torch.Generator().manual_seed(1)).to(torch.int32)
-    cache, oc = _write_both(synth.FP8_E4M3, k, v, slots, T // 16, 16, 1,
+    cache, oc = _write_both(dtype, k, v, slots, T // 16, 16, 1,
                             k_scale=[scale], v_scale=[scale * 2])
     for name in ("k_cache", "v_cache"):
         g = getattr(cache, name).cpu().numpy()
@@ -58,6 +65,27 @@ def test_int8_every_finite_fp16_pattern_and_scales():
     bs = 16
     slots = torch.arange(T, dtype=torch.int32)
     cache, oc = _write_both(synth.INT8, k, v, slots, (T + bs - 1) // bs, bs, 1)
+    for name in ("k_cache", "v_cache"):
+        assert np.array_equal(getattr(cache, name).cpu().numpy(), getattr(oc, name)), name
+    for name in ("k_scale_tok", "v_scale_tok"):
+        assert np.array_equal(bits16(getattr(cache, name).cpu()), getattr(oc, name)), name
+
+
+def test_int8_half_integer_quotients():
+    # rows whose absmax is 127 have scale 1: x = k + 1/2 is an exact tie
+    # (rint to even); other rows put x / s a hair off the half-integers
+    gen = torch.Generator().manual_seed(4)
+    half = torch.arange(-127, 127, dtype=torch.float32) + 0.5
+    rows = []
+    for r in range(64):
+        x = half[torch.randint(0, half.numel(), (128,), generator=gen)]
+        x[0] = 127.0 if r % 2 == 0 else 127.0 * (1.0 + r * 2.0 ** -11)
+        rows.append(x)
+    k = torch.stack(rows).to(torch.float16).view(-1, 1, 128)
+    v = (-k.float()).to(torch.float16)
+    T = k.shape[0]
+    slots = torch.arange(T, dtype=torch.int32)
+    cache, oc = _write_both(synth.INT8, k, v, slots, T // 16, 16, 1)
     for name in ("k_cache", "v_cache"):
         assert np.array_equal(getattr(cache, name).cpu().numpy(), getattr(oc, name)), name
     for name in ("k_scale_tok", "v_scale_tok"):
