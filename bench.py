@@ -409,7 +409,8 @@ PROFILES = {
                 ("paged_quantized_kv_quant_b200/csrc/decode.cu",
                  "paged_quantized_kv_quant_b200/csrc/common.cuh")),
     "decode5": ("decode_verify_q5_2x512k_4x256k_int8_ncu.md",
-                ("paged_quantized_kv_quant_b200/csrc/decode_tn.cu",
+                ("paged_quantized_kv_quant_b200/csrc/decode_tc.cu",
+                 "paged_quantized_kv_quant_b200/csrc/kv_stage.cuh",
                  "paged_quantized_kv_quant_b200/csrc/decode.cu",
                  "paged_quantized_kv_quant_b200/csrc/split_map.cuh",
                  "paged_quantized_kv_quant_b200/csrc/common.cuh",

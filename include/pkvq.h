@@ -121,10 +121,9 @@ PKVQ_API pkvq_status pkvq_kv_write_quant(const pkvq_cache *cache, const void *k,
 
 /*
  * Workspace bytes pkvq_paged_attn_decode needs for this shape on the
- * current device: a leading area of arrival counters (the same size for
- * every shape on a device) and the split-KV partial states (fp32 O, max and
- * sum per split).  Returns 0 on invalid arguments.  The same arguments give
- * the same size and the same split plan in pkvq_paged_attn_decode.
+ * current device (split-KV partial states: fp32 O, max and sum per split).
+ * Returns 0 on invalid arguments.  The same arguments give the same size and
+ * the same split plan in pkvq_paged_attn_decode.
  */
 PKVQ_API size_t pkvq_decode_workspace_bytes(int32_t batch, int32_t q_len, int32_t num_q_heads,
                                    int32_t max_context_len, const pkvq_cache *cache);
@@ -149,17 +148,12 @@ PKVQ_API size_t pkvq_decode_workspace_bytes(int32_t batch, int32_t q_len, int32_
  *                 The kernels split each sequence's tokens over CTAs in
  *                 proportion to its own context length, read on the device.
  *   softmax_scale scores are softmax_scale * q . k_dequantized.
-  *   workspace     device scratch of at least pkvq_decode_workspace_bytes(),
- *                 zero-filled before its first use (e.g. cudaMemset once at
- *                 allocation); every call leaves it ready for the next, of
- *                 any shape.  (The last CTA of each split sequence merges it,
- *                 found through counters that it resets.)  After a device-side
- *                 wait timeout (pkvq_device_status bit 0) zero it again.
- *                 Calls that overlap on the device must not share a workspace.
+ *   workspace     device scratch of at least pkvq_decode_workspace_bytes();
+ *                 contents need not be initialised.  Calls that overlap on
+ *                 the device must not share a workspace.
  * num_q_heads must be a multiple of num_kv_heads with a group of at most 16.
  * Up to 16 query rows per KV head (q_len x group) run on mma.sync tiles;
- * 17 to 64 rows run all rows of a KV head in one tcgen05 CTA with the keys
- * on the tensor core's M dimension, 65 to 128 with the rows on M.
+ * 17 to 128 rows run all rows of a KV head in one tcgen05 CTA.
  */
 PKVQ_API pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void *q, void *out,
                                    float *lse_out, const int32_t *block_table,
@@ -181,8 +175,7 @@ PKVQ_API pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void 
  * looks up the array's device address; make that first call before any
  * stream capture.  All calls on a device share the array: calls that may
  * overlap on the device race and must be ordered by the caller.  The array
- * is zero when the library loads and needs no clearing between calls (each
- * call returns its arrival counters to zero).
+ * needs no clearing between calls.
  */
 PKVQ_API pkvq_status pkvq_paged_attn_decode_noalloc(const pkvq_cache *cache, const void *q,
                                    void *out, float *lse_out, const int32_t *block_table,

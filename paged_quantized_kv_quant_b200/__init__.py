@@ -319,8 +319,8 @@ def paged_attn_decode(cache: PagedKVCache, q: torch.Tensor, block_table: torch.T
         if tuple(query_pos.shape) != (B, q_len):
             raise ValueError("query_pos must be [batch][q_len]")
     need = decode_workspace_bytes(cache, B, q_len, Hq, max_context_len) if B else 0
-    if workspace is None and need:   # zero-filled before its first use
-        workspace = torch.zeros(need, dtype=torch.uint8, device=q.device)
+    if workspace is None and need:   # contents need not be initialised
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     cs = cache.struct()
     opts = _opts(sliding_window, query_pos)

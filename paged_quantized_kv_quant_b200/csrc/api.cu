@@ -330,13 +330,12 @@ pkvq_status pkvq_paged_attn_decode_ex(const pkvq_cache *cache, const void *q, vo
     p.split_min_blocks = plan.split_min_blocks;
     p.split_gran = plan.split_gran;
     p.scale_log2 = softmax_scale * kLog2e;
-    // workspace: [arrival counters][partial O][partial (m, l)]
-    float *ws = reinterpret_cast<float *>(static_cast<char *>(workspace) + plan.counters_bytes);
+    // workspace: [partial O][partial (m, l)]
+    float *ws = static_cast<float *>(workspace);
     const size_t n_rows_ws = (size_t)cache->num_kv_heads * plan.row_groups * plan.num_splits *
                              plan.rows_per_cta;
     p.ws_o = plan.workspace_bytes ? ws : nullptr;
     p.ws_ml = plan.workspace_bytes ? ws + n_rows_ws * kHeadDim : nullptr;
-    p.ws_cnt = plan.fused_merge ? static_cast<int *>(workspace) : nullptr;
     p.status = status_ptr();
     if (!p.status)
         return PKVQ_ERR_CUDA;

@@ -765,41 +765,14 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
                 *reinterpret_cast<float2 *>(p.ws_ml + wrow * 2) = make_float2(M, L);
         }
     }
-    if (si.nsplit == 1 || !p.ws_cnt)
-        return;
-    // The last CTA of this (row group, KV head, sequence) to finish merges its
-    // splits: each CTA publishes its partial (fence), then counts itself in;
-    // the one that completes the count resets it for the next call and reads
-    // every partial.
-    __threadfence();
-    __syncthreads();
-    int *last = reinterpret_cast<int *>(smem);   // the tiles are idle now
-    if (threadIdx.x == 0) {
-        int *cnt = p.ws_cnt + (size_t)blockIdx.y * p.num_splits + si.first;
-        const int done = atomicAdd(cnt, 1) + 1;
-        *last = done >= si.nsplit;
-        if (done >= si.nsplit)
-            atomicExch(cnt, 0);
-    }
-    __syncthreads();
-    if (!*last)
-        return;
-    __threadfence();
-    // warp w merges rows w, w + 4, ... of this CTA's row group
-    for (int r = warp; r < RC; r += kWarps) {
-        const int rr = rg * RC + r;
-        if (rr >= p.rows)
-            break;
-        MergeRow mr;
-        mr.row0 = (size_t)blockIdx.y * p.num_splits * RC + r;
-        mr.stride = RC;
-        mr.load(p, si.first, si.nsplit, 0, lane);
-        mr.finish(p, si.first, si.nsplit, b, h, rr, lane);
-    }
 }
 
-// Merge of the split partial states by a separate kernel (the tensor-core
-// decode kernels' partials), one warp per output row.
+// Merge of the split partial states by a separate kernel, one warp per
+// output row; programmatic dependent launch lets it start while the split
+// kernel's last CTAs finish.  (A variant in which the last CTA of each
+// sequence merged its splits itself, found through arrival counters, took
+// the same time on the batch-8 x 32K workload and needed a zeroed
+// workspace.)
 template <int BS>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
 {
@@ -932,21 +905,16 @@ bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv
     // CTA for all rows, so every code is fetched and converted once; the
     // mma.sync kernel would split the rows into groups that each convert it.
     plan->tc = rows > 16 && rows <= 128;
-    // up to 64 rows: keys on the tensor core's M and 128-key tiles, so that
-    // the softmax runs one thread per key instead of one per padded row
-    plan->tn = plan->tc && rows <= 64;
     plan->nt = plan->tc ? 0 : (rows <= 8 ? 1 : 2);
     plan->rows_per_cta = plan->tc ? rows : 8 * plan->nt;
     plan->row_groups = (rows + plan->rows_per_cta - 1) / plan->rows_per_cta;
     const int max_blocks = (max_context_len + block_size - 1) / block_size;
     const int units = num_kv_heads * plan->row_groups;   // grid y: (row group, KV head)
-    // splits: tensor-core kernels in whole key tiles (64 keys with rows on M,
-    // 128 with keys on M), at least 256 keys; mma.sync kernel at least
-    // kMinBlocksPerWarp blocks per warp
-    const int tile_keys = plan->tn ? 128 : 64;
+    // splits: tensor-core kernel in whole 64-key tiles, at least 256 keys;
+    // mma.sync kernel at least kMinBlocksPerWarp blocks per warp
     const int min_blocks = plan->tc ? 256 / block_size : kWarps * kMinBlocksPerWarp;
     plan->split_min_blocks = min_blocks;
-    plan->split_gran = plan->tc ? tile_keys / block_size : 1;
+    plan->split_gran = plan->tc ? 64 / block_size : 1;
     // C CTA slots per unit, at most `ctas_per_sm` CTAs on every SM (3, or
     // what fits), all resident in one wave, each slot given about the same
     // number of blocks on the device.  Rounding the count up instead would
@@ -977,17 +945,7 @@ bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv
     const size_t partials = C > batch ? (size_t)units * C * plan->rows_per_cta *
                                             (kHeadDim + 2) * sizeof(float)
                                       : 0;
-    // The mma.sync kernel merges its own splits, counting arrivals per
-    // (unit, sequence) at the sequence's first slot.  The counters sit in a
-    // leading area of fixed size for the device (units x C <= 16 CTAs per SM
-    // whenever C > batch), ahead of the partials of every plan, so that no
-    // call's partials ever land on them: they are zero between calls.
-    plan->fused_merge = partials > 0 && !plan->tc;
-    plan->counters_bytes =
-        partials > 0 ? ((size_t)16 * device_sm_count() * sizeof(int) + 255) / 256 * 256 : 0;
-    if (plan->fused_merge && (long long)units * C > 16LL * device_sm_count())
-        return false;
-    plan->workspace_bytes = plan->counters_bytes + partials;
+    plan->workspace_bytes = partials;
     return true;
 }
 
@@ -996,9 +954,7 @@ cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_
 {
     cudaError_t e;
     const bool one = plan.nt == 1;
-    if (plan.tn)
-        e = launch_decode_tn(p, kv_dtype, stream);
-    else if (plan.tc)
+    if (plan.tc)
         e = launch_decode_tc(p, kv_dtype, kmap, vmap, stream);
     else if (kv_dtype == kKvFp8)
         e = one ? launch_bs<kKvFp8, 1>(p, kmap, vmap, stream)
@@ -1012,8 +968,8 @@ cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_
     else
         e = one ? launch_bs<kKvFp16, 1>(p, kmap, vmap, stream)
                 : launch_bs<kKvFp16, 2>(p, kmap, vmap, stream);
-    if (e != cudaSuccess || p.num_splits <= p.batch || plan.fused_merge)
-        return e;   // one slot per sequence, or the split kernel merged its own splits
+    if (e != cudaSuccess || p.num_splits <= p.batch)
+        return e;   // one slot per sequence: every CTA wrote final rows
     const long long rows_total = (long long)p.batch * p.num_kv_heads * p.rows;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((rows_total + 3) / 4));

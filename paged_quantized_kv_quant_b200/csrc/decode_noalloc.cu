@@ -17,10 +17,9 @@
 //
 // Sharing: all calls on a device use the same array.  Calls that could run at
 // the same time on the device (different streams without ordering between
-// them) race on it and must be serialized by the caller.  The array starts as
-// zeros, as a workspace must; the decode kernels write every partial they
-// later read within the same call, and each call returns its arrival counters
-// (the array's leading area) to zero, so it needs no clearing between calls.
+// them) race on it and must be serialized by the caller.  The decode kernels
+// write every scratch word they later read within the same call, so the array
+// needs no clearing between calls.
 #include "../../include/pkvq.h"
 #include "internal.h"
 

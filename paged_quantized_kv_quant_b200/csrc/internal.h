@@ -62,9 +62,6 @@ struct DecodeParams {
     float scale_log2;    // softmax_scale * log2(e)
     float *ws_o;         // [row groups x Hkv][C][rows_per_cta][128] fp32, unnormalised
     float *ws_ml;        // [row groups x Hkv][C][rows_per_cta][2] fp32 (log2 max, sum)
-    int *ws_cnt;         // arrival counters [row groups x Hkv][C] (at the first slot of
-                         // each sequence), or null: the split kernel's last CTA of a
-                         // sequence merges it; zero between calls
     uint32_t *status;
 };
 
@@ -75,9 +72,6 @@ struct DecodePlan {
     int uniform_splits, uniform_bpc;    // the assignment with equal lengths
     int split_min_blocks, split_gran;
     bool tc;                            // tensor-core kernel: all rows of a KV head in one CTA
-    bool tn;                            // ... with keys on M (17..64 rows), else rows on M
-    bool fused_merge;                   // the mma.sync kernel merges its own splits
-    size_t counters_bytes;              // the workspace's leading counter area
     size_t workspace_bytes;
 };
 
@@ -86,11 +80,10 @@ struct DecodePlan {
 bool decode_plan(int kv_dtype, int batch, int q_len, int num_q_heads, int num_kv_heads,
                  int block_size, int max_context_len, DecodePlan *plan);
 
-// The tensor-core decode kernels (all rows of a KV head in one CTA): query
-// rows on the MMA's M (65..128 rows) or keys on M (17..64 rows).
+// The tensor-core decode kernel (17..128 rows: all rows of a KV head in one
+// CTA, query rows on the MMA's M).
 cudaError_t launch_decode_tc(const DecodeParams &p, int kv_dtype, const CUtensorMap &kmap,
                              const CUtensorMap &vmap, cudaStream_t stream);
-cudaError_t launch_decode_tn(const DecodeParams &p, int kv_dtype, cudaStream_t stream);
 
 cudaError_t launch_decode(const DecodeParams &p, const DecodePlan &plan, int kv_dtype,
                           const CUtensorMap &kmap, const CUtensorMap &vmap,

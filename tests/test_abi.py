@@ -165,8 +165,7 @@ def test_verify_rows_take_the_tensor_core_plan(lib, monkeypatch):
     monkeypatch.delenv("PKVQ_DECODE_CTAS_PER_SM", raising=False)
     sms, hkv, rows, batch = 148, 4, 40, 6
     C = max(batch, sms // hkv)
-    counters = 16 * sms * 4   # the leading counter area (already a multiple of 256)
-    assert _ws(lib, batch, 5, 32, hkv, 524288) == counters + hkv * C * rows * (128 + 2) * 4
+    assert _ws(lib, batch, 5, 32, hkv, 524288) == hkv * C * rows * (128 + 2) * 4
 
 
 def test_row_counts_past_one_tile_use_row_groups(lib, monkeypatch):
@@ -177,7 +176,7 @@ def test_row_counts_past_one_tile_use_row_groups(lib, monkeypatch):
     groups = 256 // 16
     units = hkv * groups
     C = max(batch, 2 * sms // units)
-    assert _ws(lib, batch, 16, 32, hkv, 65536) == 16 * sms * 4 + units * C * 16 * (128 + 2) * 4
+    assert _ws(lib, batch, 16, 32, hkv, 65536) == units * C * 16 * (128 + 2) * 4
 
 
 def test_one_slot_per_sequence_needs_no_workspace(lib, monkeypatch):

@@ -38,7 +38,7 @@ CASES = [
     (INT8, 8, 1, [2000, 77], 4, 64),        # 32 rows
     (INT8, 16, 2, [3000, 129], 6, 16),      # 48 rows
     (FP8, 32, 4, [2500, 1], 7, 32),         # 56 rows
-    (INT8, 16, 2, [1300, 700], 8, 16),      # 64 rows: the widest keys-on-M tile
+    (INT8, 16, 2, [1300, 700], 8, 16),      # 64 rows
     (FP8, 16, 2, [900], 16, 16),            # 128 rows: one full tile
     (FP8, 32, 2, [500], 16, 16),            # 256 rows: past the tile, mma.sync row groups
 ]
@@ -255,13 +255,13 @@ def test_sharded_decode_merged_matches_oracle(world, dtype, Hq, Hkv, ctx, ql, bs
 
 
 def test_decode_workspace_reused_across_shapes():
-    # One zero-filled workspace serves calls of different shapes in turn: the
-    # arrival counters sit in a leading area that no call's partials touch,
-    # and each call returns them to zero.
-    ws = torch.zeros(48 << 20, dtype=torch.uint8, device="cuda")
+    # One workspace, never cleared and first filled with NaN patterns, serves
+    # calls of different shapes in turn: every partial a call reads it wrote
+    # itself.
+    ws = torch.full((48 << 20,), 0xFF, dtype=torch.uint8, device="cuda")
     specs = [
-        (FP8, 32, 4, [16384, 300, 5000], 1, 16),    # mma.sync, merged by its last CTAs
-        (INT8, 32, 4, [9000, 17], 5, 16),           # tcgen05 (keys on M), merge kernel
+        (FP8, 32, 4, [16384, 300, 5000], 1, 16),    # mma.sync, merge kernel
+        (INT8, 32, 4, [9000, 17], 5, 16),           # tcgen05, merge kernel
         (FP8, 16, 2, [20000, 4000], 1, 32),         # mma.sync again, other partial sizes
         (INT8, 16, 4, [3000, 12000, 64], 1, 16),
     ]
@@ -277,6 +277,4 @@ def test_decode_workspace_reused_across_shapes():
         fresh = pk.paged_attn_decode(cache, q, bt, cl, max(ctx), case.softmax_scale)
         torch.cuda.synchronize()
         assert torch.equal(shared, fresh)
-    # the counter area is back to zero
-    assert int(ws[: 16 * 148 * 4].view(torch.int32).abs().max()) == 0
     assert pk.device_status() == 0
