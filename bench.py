@@ -4,8 +4,9 @@
 One step = one decode step of the batch-8 workload (8 sequences x 32,768
 cached tokens, 32 query / 4 KV heads, head_dim 128, block 16, FP8 E4M3 cache
 with per-KV-head scales, 1% outlier channels x8): write + quantize the step's
-new token into the paged cache (pkvq_kv_write_quant), then attend over the
-whole cache (pkvq_paged_attn_decode: split kernel + merge kernel).  The metric
+new token into the paged cache and attend over the whole cache, in one call
+(pkvq_paged_attn_decode_append: the split kernel writes the new tokens of its
+blocks first, then the merge kernel).  The metric
 is KV-read GB/s: the K and V code bytes one step must read (268,435,456 B per
 GPU) divided by the step time.
 
@@ -53,7 +54,7 @@ METRIC = "paged FP8-KV attention: decode KV-read GB/s"
 def decode_config(spec, world: int):
     return {"workload": spec.name, "batch": 8, "context": 32768, "q_heads": 32,
             "kv_heads": 4, "head_dim": 128, "block_size": 16, "kv_dtype": "fp8_e4m3",
-            "step": "kv_write_quant(new token) + paged_attn_decode",
+            "step": "paged_attn_decode_append: new token's KV write + decode in one call",
             "l2": "inputs larger than L2: two 268 MB caches alternated step by step",
             "parallelism": f"dp{world} (independent batches per GPU)"}
 PREFILL_WORKLOAD = 3
@@ -351,9 +352,16 @@ def build_decode(case, device, copies: int = 2):
 
 
 def decode_step(pk, cache, inp, max_ctx, scale, write=True, decode=True):
-    if write:
+    """write and decode: one appending call; one of them alone: that call."""
+    if write and decode:
+        q = inp["q"]
+        shp = (q.shape[0], q.shape[1], cache.num_kv_heads, q.shape[3])
+        pk.paged_attn_decode_append(cache, inp["k_new"].view(shp), inp["v_new"].view(shp), q,
+                                    inp["bt"], inp["ctx"], max_ctx, scale, out=inp["out"],
+                                    workspace=inp["ws"])
+    elif write:
         pk.kv_write_quant(cache, inp["k_new"], inp["v_new"], inp["slot_new"])
-    if decode:
+    elif decode:
         pk.paged_attn_decode(cache, inp["q"], inp["bt"], inp["ctx"], max_ctx, scale,
                              out=inp["out"], workspace=inp["ws"])
 
@@ -749,12 +757,12 @@ def main():
     dec_gbs = kv_bytes / (ms_dec * 1e-3) / 1e9
 
     # ---------------- end to end through the public API, host buffers ----------------
-    # Every step uploads its inputs (new token's K/V and slots, Q, block table,
-    # context lengths) from pinned host memory and reads its output back.  The
+    # Every step uploads its inputs (new token's K/V, Q, block table, context
+    # lengths) from pinned host memory and reads its output back.  The
     # inputs sit back to back in one pinned buffer, so one copy moves them; two
     # device copies of that buffer (and of the output) let step i+1's upload
     # and step i's download run on their own streams while step i computes.
-    names = ("q", "k_new", "v_new", "slot_new", "bt", "ctx")
+    names = ("q", "k_new", "v_new", "bt", "ctx")
     offs, total = {}, 0
     for k in names:
         nb = inp[k].numel() * inp[k].element_size()
@@ -787,9 +795,10 @@ def main():
         if i >= 2:
             stream.wait_event(read[b])       # step i-2's output has been read back
         d = views[b]
-        pk.kv_write_quant(caches[i % 2], d["k_new"], d["v_new"], d["slot_new"], stream=stream)
-        pk.paged_attn_decode(caches[i % 2], d["q"], d["bt"], d["ctx"], max_ctx, scale,
-                             out=dev_out[b], workspace=inp["ws"], stream=stream)
+        shp = (d["q"].shape[0], d["q"].shape[1], caches[0].num_kv_heads, d["q"].shape[3])
+        pk.paged_attn_decode_append(caches[i % 2], d["k_new"].view(shp), d["v_new"].view(shp),
+                                    d["q"], d["bt"], d["ctx"], max_ctx, scale, out=dev_out[b],
+                                    workspace=inp["ws"], stream=stream)
         done[b].record(stream)
         down.wait_event(done[b])
         with torch.cuda.stream(down):
@@ -883,7 +892,7 @@ def main():
                 c5, oc, rows5, "GB/s", "verify decode, one 256K sequence, 5 tokens x 8 heads")
             del oc
 
-    launches_per_step = 2 + (1 if plan_splits else 0)
+    launches_per_step = 1 + (1 if plan_splits else 0)   # appending split kernel (+ merge)
     traffic = decode_traffic_from_profile()
     line = {
         "metric": METRIC,

@@ -242,6 +242,35 @@ PKVQ_API pkvq_status pkvq_paged_attn_decode_ex(const pkvq_cache *cache, const vo
                                    size_t workspace_bytes, void *stream);
 
 /*
+ * One decode step with its KV write: the step's new keys and values are
+ * quantised into the cache exactly as pkvq_kv_write_quant does, then the
+ * attention of pkvq_paged_attn_decode_ex runs over the whole context.
+ * Source: "ReVolta" PyPI page, "Weight and KV formats" (new K/V quantised
+ * into the 8-bit cache) and "1Cat-LLM" README, "Layer 1" / "Layer 2" (the
+ * decode attention); the pages run the two as separate steps, this call
+ * fuses them where it can.
+ *   k_new, v_new  fp16 [batch][q_len][num_kv_heads][head_dim]: the keys and
+ *                 values of each sequence's last q_len positions
+ *                 (context_lens[b] - q_len + t), which land in the slots the
+ *                 block table gives those positions (positions below 0 are
+ *                 skipped).  16-byte aligned.
+ * Every other argument as pkvq_paged_attn_decode_ex; opts->query_pos must
+ * be NULL (PKVQ_ERR_INVALID_ARG otherwise).  Up to 16 query rows per KV head
+ * the split-KV kernel writes the new tokens itself (the CTA that reads a
+ * token's block quantises and stores it first), so a step is one launch plus
+ * the merge; with more rows the KV write kernel runs first on the stream.
+ * The cache afterwards is bit-identical to pkvq_kv_write_quant of the same
+ * tokens, and the results to pkvq_paged_attn_decode_ex after it.
+ */
+PKVQ_API pkvq_status pkvq_paged_attn_decode_append(const pkvq_cache *cache, const void *k_new,
+                                   const void *v_new, const void *q, void *out, float *lse_out,
+                                   const int32_t *block_table, int32_t max_blocks_per_seq,
+                                   const int32_t *context_lens, int32_t batch, int32_t q_len,
+                                   int32_t num_q_heads, int32_t max_context_len,
+                                   float softmax_scale, const pkvq_attn_opts *opts,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * pkvq_paged_attn_prefill with options (sliding window; query_pos must be
  * NULL, else PKVQ_ERR_UNSUPPORTED).
  */

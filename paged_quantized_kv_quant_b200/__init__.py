@@ -37,6 +37,7 @@ _FP8_FORMATS = (KV_FP8_E4M3, KV_FP8_E5M2)
 EXPORTED = (
     "pkvq_kv_write_quant",
     "pkvq_decode_workspace_bytes",
+    "pkvq_paged_attn_decode_append",
     "pkvq_paged_attn_decode",
     "pkvq_paged_attn_decode_ex",
     "pkvq_paged_attn_decode_noalloc",
@@ -116,6 +117,9 @@ def load_library(path: Optional[str] = None) -> ctypes.CDLL:
     lib.pkvq_paged_attn_decode_ex.restype = I32
     lib.pkvq_paged_attn_decode_ex.argtypes = [P, P, P, P, P, I32, P, I32, I32, I32, I32,
                                               ctypes.c_float, P, P, SZ, P]
+    lib.pkvq_paged_attn_decode_append.restype = I32
+    lib.pkvq_paged_attn_decode_append.argtypes = [P, P, P, P, P, P, P, I32, P, I32, I32, I32,
+                                                  I32, ctypes.c_float, P, P, SZ, P]
     lib.pkvq_paged_attn_prefill.restype = I32
     lib.pkvq_paged_attn_prefill.argtypes = [P, P, P, P, P, P, I32, P, I32, I32, I32,
                                             ctypes.c_float, P, SZ, P]
@@ -329,6 +333,44 @@ def paged_attn_decode(cache: PagedKVCache, q: torch.Tensor, block_table: torch.T
         int(block_table.shape[1]), _ptr(context_lens), B, q_len, Hq, int(max_context_len),
         float(softmax_scale), None if opts is None else ctypes.byref(opts), _ptr(workspace),
         wbytes, _stream(stream)), "paged_attn_decode")
+    return out
+
+
+def paged_attn_decode_append(cache: PagedKVCache, k_new: torch.Tensor, v_new: torch.Tensor,
+                             q: torch.Tensor, block_table: torch.Tensor,
+                             context_lens: torch.Tensor, max_context_len: int,
+                             softmax_scale: float, out: Optional[torch.Tensor] = None,
+                             lse: Optional[torch.Tensor] = None,
+                             workspace: Optional[torch.Tensor] = None, stream=None,
+                             sliding_window: int = 0) -> torch.Tensor:
+    """One decode step with its KV write: k_new / v_new fp16 [B][q_len][Hkv][D]
+    are the keys and values of each sequence's last q_len positions; they are
+    quantised into the cache (as kv_write_quant) and attention runs as
+    paged_attn_decode."""
+    _need(q, torch.float16, "q", 4)
+    _need(k_new, torch.float16, "k_new", 4)
+    _need(v_new, torch.float16, "v_new", 4)
+    _need(block_table, torch.int32, "block_table", 2)
+    _need(context_lens, torch.int32, "context_lens", 1)
+    B, q_len, Hq, D = q.shape
+    if tuple(k_new.shape) != (B, q_len, cache.num_kv_heads, D) or k_new.shape != v_new.shape:
+        raise ValueError("k_new / v_new must be [batch][q_len][num_kv_heads][head_dim]")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, torch.float16, "out", 4)
+    if lse is not None:
+        _need(lse, torch.float32, "lse", 3)
+    need = decode_workspace_bytes(cache, B, q_len, Hq, max_context_len) if B else 0
+    if workspace is None and need:   # contents need not be initialised
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    cs = cache.struct()
+    opts = _opts(sliding_window, None)
+    _check(_lib().pkvq_paged_attn_decode_append(
+        ctypes.byref(cs), _ptr(k_new), _ptr(v_new), _ptr(q), _ptr(out), _ptr(lse),
+        _ptr(block_table), int(block_table.shape[1]), _ptr(context_lens), B, q_len, Hq,
+        int(max_context_len), float(softmax_scale), None if opts is None else ctypes.byref(opts),
+        _ptr(workspace), wbytes, _stream(stream)), "paged_attn_decode_append")
     return out
 
 

@@ -252,13 +252,16 @@ pkvq_status pkvq_paged_attn_decode(const pkvq_cache *cache, const void *q, void 
                                      softmax_scale, nullptr, workspace, workspace_bytes, stream);
 }
 
-pkvq_status pkvq_paged_attn_decode_ex(const pkvq_cache *cache, const void *q, void *out,
-                                      float *lse_out, const int32_t *block_table,
-                                      int32_t max_blocks_per_seq, const int32_t *context_lens,
-                                      int32_t batch, int32_t q_len, int32_t num_q_heads,
-                                      int32_t max_context_len, float softmax_scale,
-                                      const pkvq_attn_opts *opts, void *workspace,
-                                      size_t workspace_bytes, void *stream)
+namespace {
+
+// Decode, optionally appending the step's new tokens (k_new / v_new: the
+// keys and values of each sequence's last q_len positions) first.
+pkvq_status decode_impl(const pkvq_cache *cache, const void *k_new, const void *v_new,
+                        const void *q, void *out, float *lse_out, const int32_t *block_table,
+                        int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t batch,
+                        int32_t q_len, int32_t num_q_heads, int32_t max_context_len,
+                        float softmax_scale, const pkvq_attn_opts *opts, void *workspace,
+                        size_t workspace_bytes, void *stream)
 {
     if (opts && opts->sliding_window < 0)
         return PKVQ_ERR_INVALID_ARG;
@@ -339,7 +342,79 @@ pkvq_status pkvq_paged_attn_decode_ex(const pkvq_cache *cache, const void *q, vo
     p.status = status_ptr();
     if (!p.status)
         return PKVQ_ERR_CUDA;
-    return from_cuda(launch_decode(p, plan, cache->dtype, km, vm, static_cast<cudaStream_t>(stream)));
+    cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+    if (k_new) {
+        if (plan.tc) {
+            // the tensor-core kernel reads whole tiles through one copy ring:
+            // the new tokens are written by the KV write kernel just before
+            KvWriteParams w{};
+            w.k_cache = static_cast<uint8_t *>(cache->k_cache);
+            w.v_cache = static_cast<uint8_t *>(cache->v_cache);
+            w.k_scale = cache->k_scale;
+            w.v_scale = cache->v_scale;
+            w.scale_stride = scale_stride(cache);
+            w.k_scale_tok = static_cast<uint16_t *>(cache->k_scale_tok);
+            w.v_scale_tok = static_cast<uint16_t *>(cache->v_scale_tok);
+            w.k = static_cast<const __half *>(k_new);
+            w.v = static_cast<const __half *>(v_new);
+            w.slot_mapping = nullptr;
+            w.block_table = block_table;
+            w.context_lens = context_lens;
+            w.max_blocks_per_seq = max_blocks_per_seq;
+            w.q_len = q_len;
+            w.num_tokens = batch * q_len;
+            w.num_kv_heads = cache->num_kv_heads;
+            w.num_blocks = cache->num_blocks;
+            w.block_size = cache->block_size;
+            w.status = p.status;
+            const cudaError_t e = launch_kv_write_quant(w, cache->dtype, st_);
+            if (e != cudaSuccess)
+                return from_cuda(e);
+        } else {
+            // the split kernel: each CTA writes the new tokens of its blocks
+            p.k_new = static_cast<const __half *>(k_new);
+            p.v_new = static_cast<const __half *>(v_new);
+        }
+    }
+    return from_cuda(launch_decode(p, plan, cache->dtype, km, vm, st_));
+}
+
+}  // namespace
+
+pkvq_status pkvq_paged_attn_decode_ex(const pkvq_cache *cache, const void *q, void *out,
+                                      float *lse_out, const int32_t *block_table,
+                                      int32_t max_blocks_per_seq, const int32_t *context_lens,
+                                      int32_t batch, int32_t q_len, int32_t num_q_heads,
+                                      int32_t max_context_len, float softmax_scale,
+                                      const pkvq_attn_opts *opts, void *workspace,
+                                      size_t workspace_bytes, void *stream)
+{
+    return decode_impl(cache, nullptr, nullptr, q, out, lse_out, block_table,
+                       max_blocks_per_seq, context_lens, batch, q_len, num_q_heads,
+                       max_context_len, softmax_scale, opts, workspace, workspace_bytes, stream);
+}
+
+pkvq_status pkvq_paged_attn_decode_append(const pkvq_cache *cache, const void *k_new,
+                                          const void *v_new, const void *q, void *out,
+                                          float *lse_out, const int32_t *block_table,
+                                          int32_t max_blocks_per_seq,
+                                          const int32_t *context_lens, int32_t batch,
+                                          int32_t q_len, int32_t num_q_heads,
+                                          int32_t max_context_len, float softmax_scale,
+                                          const pkvq_attn_opts *opts, void *workspace,
+                                          size_t workspace_bytes, void *stream)
+{
+    if (opts && opts->query_pos)
+        return PKVQ_ERR_INVALID_ARG;   // the new tokens are the last q_len positions
+    if (batch > 0) {
+        if (!k_new || !v_new)
+            return PKVQ_ERR_INVALID_ARG;
+        if (!aligned16(k_new) || !aligned16(v_new))
+            return PKVQ_ERR_MISALIGNED;
+    }
+    return decode_impl(cache, k_new, v_new, q, out, lse_out, block_table, max_blocks_per_seq,
+                       context_lens, batch, q_len, num_q_heads, max_context_len, softmax_scale,
+                       opts, workspace, workspace_bytes, stream);
 }
 
 pkvq_status pkvq_paged_attn_prefill(const pkvq_cache *cache, const void *q, void *out,

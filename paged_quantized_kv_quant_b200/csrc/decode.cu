@@ -43,6 +43,7 @@
 // or given per query (a rank holding part of each sequence's keys).
 #include "common.cuh"
 #include "internal.h"
+#include "quant.cuh"
 #include "split_map.cuh"
 
 #include <math.h>
@@ -306,6 +307,51 @@ __device__ __forceinline__ void pv_block_f16(const uint8_t *vt, int g, int t, in
     }
 }
 
+// The step's new tokens (each sequence's last q_len positions) that fall in
+// positions [lo_pos, hi_pos): their K and V rows of KV head h quantised and
+// stored in the cache exactly as the KV write kernel does, 16 threads (a
+// half-warp) per token and 8 tokens per pass.
+template <int KVT, int BS>
+__device__ __forceinline__ void append_tokens(const DecodeParams &p, int b, int h, int ctx,
+                                              int lo_pos, int hi_pos, const int32_t *bt)
+{
+    const int grp = threadIdx.x >> 4, sub = threadIdx.x & 15;
+    uint8_t *kc = const_cast<uint8_t *>(p.k_cache);
+    uint8_t *vc = const_cast<uint8_t *>(p.v_cache);
+    uint16_t *kst = const_cast<uint16_t *>(p.k_scale_tok);
+    uint16_t *vst = const_cast<uint16_t *>(p.v_scale_tok);
+    float ks = 0.0f, vs = 0.0f;
+    if constexpr (kv_has_head_scale(KVT)) {
+        ks = __ldg(p.k_scale + h * p.scale_stride);
+        vs = __ldg(p.v_scale + h * p.scale_stride);
+    }
+    for (int t0 = 0; t0 < p.q_len; t0 += kThreads / 16) {   // the same passes on every thread
+        const int t = t0 + grp;
+        const int pos = ctx - p.q_len + t;
+        bool mine = t < p.q_len && pos >= 0 && pos >= lo_pos && pos < hi_pos &&
+                    pos / BS < p.max_blocks_per_seq;
+        int phys = mine ? __ldg(bt + pos / BS) : 0;
+#ifdef PKVQ_BOUNDS_CHECK
+        if (mine && (phys < 0 || phys >= p.num_blocks)) {
+            if (sub == 0)
+                atomicOr(p.status, kStatusBadBlock);
+            mine = false;
+            phys = 0;
+        }
+#endif
+        const size_t drow = ((size_t)phys * p.num_kv_heads + h) * BS + (mine ? pos % BS : 0);
+        uint4 kx = make_uint4(0u, 0u, 0u, 0u), vx = kx;
+        if (mine) {
+            const size_t src =
+                (((size_t)b * p.q_len + t) * p.num_kv_heads + h) * kHeadDim + sub * 8;
+            kx = __ldg(reinterpret_cast<const uint4 *>(p.k_new + src));
+            vx = __ldg(reinterpret_cast<const uint4 *>(p.v_new + src));
+        }
+        quant_store_piece<KVT>(kc, kst, ks, drow, sub, kx, mine);
+        quant_store_piece<KVT>(vc, vst, vs, drow, sub, vx, mine);
+    }
+}
+
 // Merge of the split partial states of one output row by one warp:
 // M = max_i m_i, L = sum_i l_i 2^(m_i - M), O = sum_i O_i 2^(m_i - M) / L.
 // The splits are taken kMergeChunk at a time: every lane issues the loads of
@@ -490,6 +536,14 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
     const int nblk = max(0, min(nblk_seq, blk_begin + si.bpc) - blk_begin);
     const int n_it = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
     const int32_t *bt = p.block_table + (size_t)b * p.max_blocks_per_seq;
+    // Appending call: the step's new tokens in this CTA's blocks are
+    // quantised and stored first (no other CTA of this KV head reads those
+    // slots), then made visible to the tensor copies below.
+    if (p.k_new) {
+        append_tokens<KVT, BS>(p, b, h, ctx, blk_begin * BS, (blk_begin + nblk) * BS, bt);
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncthreads();
+    }
     // each thread's two rows per n8 tile: last visible key (pos) and first
     // (lo); padding rows see the whole split
     int pos[NT][2], lo[NT][2];

@@ -30,7 +30,10 @@ struct KvWriteParams {
     int scale_stride;                      // 1: per KV head; 0: one scale per layer
     uint16_t *k_scale_tok, *v_scale_tok;   // INT8 (fp16 bits)
     const __half *k, *v;
-    const int32_t *slot_mapping;
+    const int32_t *slot_mapping;   // or null: the slots of each sequence's last q_len
+                                   // positions, from block_table and context_lens
+    const int32_t *block_table, *context_lens;
+    int max_blocks_per_seq, q_len;
     int num_tokens, num_kv_heads, num_blocks, block_size;
     uint32_t *status;
 };
@@ -39,6 +42,9 @@ cudaError_t launch_kv_write_quant(const KvWriteParams &p, int kv_dtype, cudaStre
 
 struct DecodeParams {
     const uint8_t *k_cache, *v_cache;            // [blocks][Hkv][block_size][row bytes]
+    const __half *k_new, *v_new;                 // nullable [batch][q_len][Hkv][128]: the
+                                                 // split kernel writes these new tokens
+                                                 // (the last q_len positions) first
     const float *k_scale, *v_scale;              // FP8 formats: per KV head (or layer)
     int scale_stride;                            // 1: per KV head; 0: one per layer
     const uint16_t *k_scale_tok, *v_scale_tok;   // INT8: per (block, head, token)
