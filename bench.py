@@ -18,7 +18,7 @@ bf16 tensor peak), the 2 x 512K + 4 x 256K INT8 verify decode (KV GB/s
 against HBM), and the KV writes of the two prefills.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pkvq|reference]
-    python bench.py --only decode|prefill [--workload n] [--steps K] [--warmup W]
+    python bench.py --only decode|prefill|kv_write [--workload n] [--steps K] [--warmup W]
 
 --only runs nothing but W + K calls of one kernel path on its workload and
 prints their average time: the command the ncu captures are taken with.
@@ -75,9 +75,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip every secondary workload")
-    ap.add_argument("--only", choices=["decode", "prefill"], default=None)
+    ap.add_argument("--only", choices=["decode", "prefill", "kv_write"], default=None)
     ap.add_argument("--workload", type=int, default=None,
-                    help="with --only: the named workload to run (decode 1, 2, 5; prefill 3, 4)")
+                    help="with --only: the named workload to run (decode 1, 2, 5; prefill "
+                         "and kv_write 3, 4)")
     ap.add_argument("--ctx-div", type=int, default=1,
                     help="with --only decode: divide every context length by this (a smaller "
                          "case of the same shape, e.g. for a profiler capture)")
@@ -415,7 +416,9 @@ def time_graph(graph, reps, stream, barrier=None):
 PROFILES = {
     "decode2": ("decode_b8_ctx32k_fp8_ncu.md",
                 ("paged_quantized_kv_quant_b200/csrc/decode.cu",
-                 "paged_quantized_kv_quant_b200/csrc/common.cuh")),
+                 "paged_quantized_kv_quant_b200/csrc/common.cuh",
+                 "paged_quantized_kv_quant_b200/csrc/quant.cuh",
+                 "paged_quantized_kv_quant_b200/csrc/split_map.cuh")),
     "decode5": ("decode_verify_q5_2x512k_4x256k_int8_ncu.md",
                 ("paged_quantized_kv_quant_b200/csrc/decode_tc.cu",
                  "paged_quantized_kv_quant_b200/csrc/kv_stage.cuh",
@@ -423,9 +426,13 @@ PROFILES = {
                  "paged_quantized_kv_quant_b200/csrc/split_map.cuh",
                  "paged_quantized_kv_quant_b200/csrc/common.cuh",
                  "paged_quantized_kv_quant_b200/csrc/tc.cuh")),
+    "kvwrite4": ("kv_write_131k_fp8_ncu.md",
+                 ("paged_quantized_kv_quant_b200/csrc/kv_write.cu",
+                  "paged_quantized_kv_quant_b200/csrc/quant.cuh")),
     "prefill3": ("prefill_8k_causal_fp8_ncu.md",
                  ("paged_quantized_kv_quant_b200/csrc/prefill_tc.cu",
                   "paged_quantized_kv_quant_b200/csrc/common.cuh",
+                  "paged_quantized_kv_quant_b200/csrc/kv_stage.cuh",
                   "paged_quantized_kv_quant_b200/csrc/tc.cuh")),
 }
 DECODE_PROFILE = os.path.join(ROOT, "profiles", PROFILES["decode2"][0])
@@ -503,6 +510,15 @@ def run_only(args):
         torch.cuda.empty_cache()   # keep only what the calls use on the device
         calls = [lambda c=c: decode_step(pk, c, inp, max_ctx, case.softmax_scale, write=False)
                  for c in caches]
+    elif args.only == "kv_write":
+        # the KV write of every cached token of a prefill workload, as the
+        # prefill secondaries time it
+        spec = synth.workload(args.workload or PREFILL_WORKLOAD)
+        case = synth.make_case(spec)
+        c = new_cache(pk, case, device)
+        kd, vd = case.k.to(device), case.v.to(device)
+        smd = case.slot_mapping.to(device)
+        calls = [lambda: pk.kv_write_quant(c, kd, vd, smd)]
     else:
         spec = synth.workload(args.workload or PREFILL_WORKLOAD)
         case = synth.make_case(spec)
@@ -598,7 +614,8 @@ def sec_prefill(pk, n, device, stream, clk, bf16_peak, hbm_peak, peak_src):
               "unit": "GB/s", "ms": ms_wr, "timed_calls": reps_wr, "bytes": wbytes,
               "frac": wgbs / hbm_peak,
               "roofline": {"bound": "hbm", "achieved": wgbs, "peak": hbm_peak, "unit": "GB/s",
-                           "frac": wgbs / hbm_peak, "peak_source": peak_src, "traffic": None}}
+                           "frac": wgbs / hbm_peak, "peak_source": peak_src,
+                           "traffic": traffic_from_profile("kvwrite4") if n == 4 else None}}
     del g_pf, g_wr, c, kd, vd, smd, q, out
     torch.cuda.empty_cache()
     return entry, wentry, case

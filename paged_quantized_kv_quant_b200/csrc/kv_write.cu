@@ -21,10 +21,11 @@ constexpr int kD = 128;
 constexpr int kThreadsPerRow = 16;
 constexpr int kElemsPerThread = 8;
 constexpr int kBlockThreads = 256;
-constexpr int kGroupsPerBlock = kBlockThreads / kThreadsPerRow;
-constexpr int kRowsPerBlock = kGroupsPerBlock;
+constexpr int kTokensPerBlock = kBlockThreads / kThreadsPerRow;
 
-template <int KVT>
+// Grid: x = token groups of 16, y = KV head, so that no thread divides by a
+// run-time value (the block size is a template parameter).
+template <int KVT, int BS>
 __global__ void __launch_bounds__(kBlockThreads)
 kv_write_quant_kernel(KvWriteParams p)
 {
@@ -33,11 +34,10 @@ kv_write_quant_kernel(KvWriteParams p)
     // finish before it reads anything.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int sub = threadIdx.x % kThreadsPerRow;
-    const long long nrows = (long long)p.num_tokens * p.num_kv_heads;
-    const long long row = (long long)blockIdx.x * kRowsPerBlock + threadIdx.x / kThreadsPerRow;
-    const bool active = row < nrows;
-    const int tok = active ? (int)(row / p.num_kv_heads) : 0;
-    const int h = active ? (int)(row % p.num_kv_heads) : 0;
+    const int h = blockIdx.y;
+    const long long tl = (long long)blockIdx.x * kTokensPerBlock + threadIdx.x / kThreadsPerRow;
+    const bool active = tl < p.num_tokens;
+    const int tok = active ? (int)tl : 0;
     int slot = -1;
     if (active) {
         if (p.slot_mapping) {
@@ -47,14 +47,14 @@ kv_write_quant_kernel(KvWriteParams p)
             // position ctx - q_len + t, in the block the table gives it
             const int b = tok / p.q_len, t = tok % p.q_len;
             const int pos = __ldg(p.context_lens + b) - p.q_len + t;
-            if (pos >= 0 && pos / p.block_size < p.max_blocks_per_seq)
-                slot = __ldg(p.block_table + (size_t)b * p.max_blocks_per_seq +
-                             pos / p.block_size) * p.block_size + pos % p.block_size;
+            if (pos >= 0 && pos / BS < p.max_blocks_per_seq)
+                slot = __ldg(p.block_table + (size_t)b * p.max_blocks_per_seq + pos / BS) * BS +
+                       pos % BS;
         }
     }
     bool write = slot >= 0;
 #ifdef PKVQ_BOUNDS_CHECK
-    if (write && (long long)slot >= (long long)p.num_blocks * p.block_size) {
+    if (write && (long long)slot >= (long long)p.num_blocks * BS) {
         if (sub == 0)
             atomicOr(p.status, kStatusBadBlock);
         write = false;
@@ -68,9 +68,9 @@ kv_write_quant_kernel(KvWriteParams p)
         kx = __ldcs(reinterpret_cast<const uint4 *>(p.k + src));
         vx = __ldcs(reinterpret_cast<const uint4 *>(p.v + src));
     }
-    const int blk = write ? slot / p.block_size : 0;
-    const int off = write ? slot % p.block_size : 0;
-    const size_t drow = ((size_t)blk * p.num_kv_heads + h) * p.block_size + off;
+    const int blk = write ? slot / BS : 0;
+    const int off = write ? slot % BS : 0;
+    const size_t drow = ((size_t)blk * p.num_kv_heads + h) * BS + off;
     float ks = 0.0f, vs = 0.0f;
     if constexpr (kv_has_head_scale(KVT)) {
         if (write) {
@@ -82,22 +82,33 @@ kv_write_quant_kernel(KvWriteParams p)
     quant_store_piece<KVT>(p.v_cache, p.v_scale_tok, vs, drow, sub, vx, write);
 }
 
+template <int KVT>
+cudaError_t launch_kw(const KvWriteParams &p, dim3 grid, cudaStream_t stream)
+{
+    switch (p.block_size) {
+    case 16: kv_write_quant_kernel<KVT, 16><<<grid, kBlockThreads, 0, stream>>>(p); break;
+    case 32: kv_write_quant_kernel<KVT, 32><<<grid, kBlockThreads, 0, stream>>>(p); break;
+    case 64: kv_write_quant_kernel<KVT, 64><<<grid, kBlockThreads, 0, stream>>>(p); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_kv_write_quant(const KvWriteParams &p, int kv_dtype, cudaStream_t stream)
 {
-    const long long nrows = (long long)p.num_tokens * p.num_kv_heads;
-    if (nrows == 0)
+    if (p.num_tokens == 0 || p.num_kv_heads == 0)
         return cudaSuccess;
-    const unsigned grid = (unsigned)((nrows + kRowsPerBlock - 1) / kRowsPerBlock);
+    const dim3 grid((unsigned)((p.num_tokens + kTokensPerBlock - 1) / kTokensPerBlock),
+                    (unsigned)p.num_kv_heads);
     switch (kv_dtype) {
-    case kKvFp8: kv_write_quant_kernel<kKvFp8><<<grid, kBlockThreads, 0, stream>>>(p); break;
-    case kKvInt8: kv_write_quant_kernel<kKvInt8><<<grid, kBlockThreads, 0, stream>>>(p); break;
-    case kKvE5m2: kv_write_quant_kernel<kKvE5m2><<<grid, kBlockThreads, 0, stream>>>(p); break;
-    case kKvFp16: kv_write_quant_kernel<kKvFp16><<<grid, kBlockThreads, 0, stream>>>(p); break;
+    case kKvFp8: return launch_kw<kKvFp8>(p, grid, stream);
+    case kKvInt8: return launch_kw<kKvInt8>(p, grid, stream);
+    case kKvE5m2: return launch_kw<kKvE5m2>(p, grid, stream);
+    case kKvFp16: return launch_kw<kKvFp16>(p, grid, stream);
     default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace pkvq
