@@ -18,29 +18,34 @@
 // tile, tensor memory holds two S buffers: S(j+2) = Q K(j+2)^T is issued as
 // soon as P(j) V has been, and the softmax finds its next S ready.
 //
-// Warp roles (12 warps; the softmax warps form one aligned group of four, as
+// Warp roles (14 warps; the softmax warps form one aligned group of four, as
 // each warp reaches only the tensor-memory lanes 32 * (warp % 4) + 0..31):
-//   warps 0-3, 6-7  dequant: code tiles -> fp16 K/V tiles in the
-//              128-byte-swizzled layout [d half][key][64 d] (the K-major B
-//              operand of Q K^T and the MN-major B operand of P V), one key
-//              row per thread: warps 0-1 convert d 0-63 of K, warps 6-7 d
-//              64-127 of K, warps 2-3 all of V.  With one query tile nothing
-//              else shares the conversion of a tile, so it takes six warps to
-//              keep pace with the softmax; K is split further because Q K^T
-//              of a tile waits for it.
-//   warp 4     TMA producer: one 2-D box per cache block into a 5-stage ring.
-//   warp 5     TMEM allocation; the whole warp runs the issue loop, one
+//   warps 0-7  dequant: code tiles -> fp16 K/V tiles in the 128-byte-
+//              swizzled layout [d half][key][64 d] (the K-major B operand of
+//              Q K^T and the MN-major B operand of P V).  Warps 0-3 convert
+//              K, warps 4-7 V, each one 32-key half of a tile and one d half
+//              (64 codes per thread and tile), so every SM sub-partition runs
+//              one K and one V warp.  Each thread copies its own 64 code bytes
+//              into a 5-stage ring with 16-byte cp.async four tiles ahead and
+//              reads back only those: no producer warp issues the ~1,000
+//              copies of a tile alone, and no barrier hands the codes over.
+//   warp 8     TMEM allocation; the whole warp runs the issue loop, one
 //              elected lane issues each tcgen05 instruction.
-//   warps 8-11 softmax, thread i owns row i: Q row into tensor memory, S row
-//              read with tcgen05.ld, causal mask where a tile can cross a
-//              row's position, FP32 running max/sum, fp16 P row written over
-//              its S columns, lazy O rescale.
+//   warp 9     L2 prefetch of the tiles up to kPrefetchTiles ahead of the
+//              conversion (FP16 caches: also the copies, see below).
+//   warps 10-13 softmax: Q rows into tensor memory, S read with tcgen05.ld,
+//              causal mask where a tile can cross a row's position, FP32
+//              running max/sum, fp16 P written over its S columns, lazy O
+//              rescale.  Up to 64 rows, row 4 i + q sits in lane i of quadrant
+//              q and each such lane's scores are split over two threads
+//              (16x32bx2 tensor-memory loads): exponentials of padding lanes
+//              are never computed.  Beyond 64 rows each thread owns one row.
 // Epilogue: the final fp16 row when one split covers the sequence, otherwise
 // an FP32 partial (unnormalised O, max in log2 units, sum) in the decode
 // workspace, which the decode merge kernel combines.
 //
-// FP16 caches need no conversion: the TMA warp copies each block's two
-// 128-byte row halves straight into a K/V buffer (the same swizzled layout),
+// FP16 caches need no conversion: warp 9 copies each key's two 128-byte row
+// halves straight into a K/V buffer (the same swizzled layout) with cp.async,
 // and the dequant warps only clear the rows past the context or the split
 // before releasing the buffer to the MMA warp (never-written slots may hold
 // NaN patterns, and 0 * NaN in P V would poison O).
@@ -56,40 +61,47 @@
 namespace pkvq {
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 448;
 constexpr int kKT = 64;              // keys per tile
-// 5 code stages (80 KB per SM in flight) and 4 K/V buffers: issuing Q K^T
-// two tiles ahead holds tiles j, j+1 and j+2, and the fourth lets the
-// dequantisation of j+3 start before P(j) V has completed.
-constexpr int kCodeStages = 5;
+// 4 K/V buffers: issuing Q K^T two tiles ahead holds tiles j, j+1 and j+2,
+// and the fourth lets the dequantisation of j+3 start before P(j) V has
+// completed.
 constexpr int kKVBufs = 4;
-// L2 prefetch distance in tiles: with 16-token blocks the farthest prefetched
-// block stays within 60 entries of the block-table window's base
+// L2 prefetch distance in tiles (~100 KB per SM in flight for 8-bit K/V):
+// with 16-token blocks the farthest prefetched block stays within 60 entries
+// of the block-table window's base
 constexpr int kPrefetchTiles = 6;
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by > 2^8
-constexpr int kWarpTma = 4;
-constexpr int kWarpMma = 5;
-constexpr int kDequantWarps = 6;   // warps 0-3 and 6-7
-
-__device__ __forceinline__ bool is_dequant_warp(int w) { return w < 4 || w == 6 || w == 7; }
-constexpr int kSoftmaxWarp0 = 8;
+constexpr int kDequantWarps = 8;   // warps 0-7
+constexpr int kWarpMma = 8;
+constexpr int kWarpPf = 9;         // L2 prefetch (FP16: the copies)
+constexpr int kSoftmaxWarp0 = 10;  // warps 10-13: lane quadrants 2, 3, 0, 1
 
 // tensor memory: S/P buffers 0 and 1 (P in the first 32 columns of its
 // buffer), O, Q (two fp16 per column)
-constexpr uint32_t kTmS = 0, kTmO = 128, kTmQ = 256;
+constexpr int kSBufs = 2;
+constexpr uint32_t kTmS = 0, kTmO = kSBufs * 64, kTmQ = kTmO + 128;
+static_assert(kTmQ + 64 <= 512, "tensor memory columns");
+__device__ __forceinline__ int sbuf(int j) { return j % kSBufs; }
+__device__ __forceinline__ uint32_t sphase(int j) { return (uint32_t)(j / kSBufs) & 1u; }
 
 // shared-memory map (offsets from a 1024-byte aligned base)
 constexpr int kOffKV = 0;                                 // bufs x (K 8K+8K, V 8K+8K)
 constexpr int kKVBuf = 32768;
-constexpr int kOffCodes = kOffKV + kKVBufs * kKVBuf;      // stages x (K 8K, V 8K)
+// 8-bit codes: a ring of kCodeStages stages (K 8K, V 8K; rows 128-byte
+// swizzled), each dequant thread copying and reading back only its own bytes;
+// copies run kCodeStages - 1 tiles ahead of the conversion
+constexpr int kCodeStages = 5;
+constexpr int kOffCodes = kOffKV + kKVBufs * kKVBuf;
 constexpr int kCodeStage = 16384;
-constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // stages x (K 64, V 64) halves
-constexpr int kOffKsf = kOffScl + kCodeStages * 256;            // bufs x 64 fp32 K factors
+constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // stages x 8 warps x 32 halves
+constexpr int kOffKsf = kOffScl + kCodeStages * kDequantWarps * 64;   // bufs x 64 fp32 K factors
 constexpr int kOffBars = kOffKsf + kKVBufs * 64 * 4;
-constexpr int kNumBars = 1 + 2 * kCodeStages + 3 * kKVBufs + 3 * 2 + 1;
+constexpr int kNumBars = 1 + 3 * kKVBufs + 3 * kSBufs + 1;
 constexpr int kOffTaddr = kOffBars + kNumBars * 8;
-constexpr int kSmemBytes = kOffTaddr + 16;
+constexpr int kOffProgress = kOffTaddr + 8;   // tiles dequantised so far (prefetch pacing)
+constexpr int kSmemBytes = kOffProgress + 8;
 constexpr size_t kSmemAlloc = kSmemBytes + 1024;
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
 
@@ -98,7 +110,6 @@ constexpr uint32_t kIdescPV = idesc_f16_f32(128, 128, true);
 
 struct Bars {
     uint64_t *q_full;
-    uint64_t *code_full, *code_empty;   // [kCodeStages]
     uint64_t *kv_full, *kv_empty;       // [kKVBufs]
     uint64_t *s_full, *p_full, *pv_done;   // [S/P buffer]
     uint64_t *mma_done;
@@ -110,14 +121,12 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *smem)
     uint64_t *b = reinterpret_cast<uint64_t *>(smem + kOffBars);
     Bars r;
     r.q_full = b;
-    r.code_full = b + 1;
-    r.code_empty = r.code_full + kCodeStages;
-    r.kv_full = r.code_empty + kCodeStages;
+    r.kv_full = b + 1;
     r.kv_empty = r.kv_full + kKVBufs;
     r.s_full = r.kv_empty + kKVBufs;
-    r.p_full = r.s_full + 2;
-    r.pv_done = r.p_full + 2;
-    r.mma_done = r.pv_done + 2;
+    r.p_full = r.s_full + kSBufs;
+    r.pv_done = r.p_full + kSBufs;
+    r.mma_done = r.pv_done + kSBufs;
     r.kv_tma = r.mma_done + 1;
     return r;
 }
@@ -145,7 +154,7 @@ __device__ __forceinline__ void cvt4(uint32_t x, uint32_t &lo, uint32_t &hi)
         s8x4_to_half2x2(x, lo, hi);
 }
 
-template <int KVT, int BS>
+template <int KVT, int BS, bool kHalf>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                  const __grid_constant__ CUtensorMap vmap, const DecodeParams p)
@@ -165,16 +174,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
 
     if (tid == 0) {
         mbar_init(bars.q_full, 4);
-        for (int s = 0; s < kCodeStages; ++s) {
-            mbar_init(&bars.code_full[s], 32);   // one cp.async arrival per producer lane
-            mbar_init(&bars.code_empty[s], kDequantWarps);
-        }
+        *reinterpret_cast<volatile int *>(smem + kOffProgress) = 0;
         for (int i = 0; i < kKVBufs; ++i) {
             mbar_init(&bars.kv_full[i], kDequantWarps);
             mbar_init(&bars.kv_empty[i], 1);
             mbar_init(&bars.kv_tma[i], 32);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kSBufs; ++i) {
             mbar_init(&bars.s_full[i], 1);
             mbar_init(&bars.p_full[i], 4);
             mbar_init(&bars.pv_done[i], 1);
@@ -210,11 +216,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     tc_fence_after();
     const uint32_t tmem = *taddr_smem;
 
-    if (warp == kWarpTma) {
-        // ---------------------------------------------- copy producer --
-        // 16-byte cp.async copies by all 32 lanes; each lane arrives on the
-        // tile's barrier once its own copies have landed.  The tiles up to
-        // kPrefetchTiles past the one being loaded are first fetched into L2.
+    if (warp == kWarpPf) {
+        // -------------------------------------------- L2 prefetch / copies --
         const CacheView cv{p.k_cache, p.v_cache, p.k_scale_tok, p.v_scale_tok, p.num_kv_heads,
                            p.num_blocks, p.status};
         BlockWindow w;
@@ -222,85 +225,111 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         // than the row can address (a caller error: those keys read block 0)
         w.init(p.block_table + (size_t)b * p.max_blocks_per_seq + blk_begin,
                min(nblk, p.max_blocks_per_seq - blk_begin), lane);
-        // FP16: each tile goes straight into K/V buffer j % kKVBufs
-        constexpr int kRing = KVT == kKvFp16 ? kKVBufs : kCodeStages;
-        int pf_next = kRing;
-        for (int j = 0; j < ntiles; ++j) {
-            for (; pf_next < ntiles && pf_next <= j + kPrefetchTiles; ++pf_next)
-                prefetch_blocks<BS, KVT>(cv, h, w, pf_next * kBPT,
-                                         min(kBPT, nblk - pf_next * kBPT), lane);
-            const int s = j % kRing;
-            uint64_t *empty = KVT == kKvFp16 ? bars.kv_empty : bars.code_empty;
-            if (j >= kRing && !warp_wait(&empty[s], ((j - kRing) / kRing) & 1, p.status))
-                break;
-            const int blk0 = j * kBPT;   // within this split
-            const int nb = min(kBPT, nblk - blk0);
-            if constexpr (KVT == kKvFp16) {
+        if constexpr (KVT == kKvFp16) {
+            // FP16 needs no conversion: 16-byte cp.async copies by all 32
+            // lanes go straight into K/V buffer j % kKVBufs, and each lane
+            // arrives on the buffer's barrier once its own copies have landed.
+            // The tiles up to kPrefetchTiles past the one being copied are
+            // first fetched into L2.
+            int pf_next = kKVBufs;
+            for (int j = 0; j < ntiles; ++j) {
+                for (; pf_next < ntiles && pf_next <= j + kPrefetchTiles; ++pf_next)
+                    prefetch_blocks<BS, KVT>(cv, h, w, pf_next * kBPT,
+                                             min(kBPT, nblk - pf_next * kBPT), lane);
+                const int s = j % kKVBufs;
+                if (j >= kKVBufs &&
+                    !warp_wait(&bars.kv_empty[s], ((j - kKVBufs) / kKVBufs) & 1, p.status))
+                    break;
+                const int blk0 = j * kBPT;   // within this split
                 const uint32_t kv = sbase + kOffKV + s * kKVBuf;
-                copy_fp16_rows<BS>(kv, kv + 16384, 8192, cv, h, w, blk0, nb, kKT, lane);
+                copy_fp16_rows<BS>(kv, kv + 16384, 8192, cv, h, w, blk0,
+                                   min(kBPT, nblk - blk0), kKT, lane);
                 cp_async_mbar_arrive(&bars.kv_tma[s]);
-            } else {
-                const uint32_t dst = sbase + kOffCodes + s * kCodeStage;
-                copy_code_rows<BS>(dst, dst + 8192, cv, h, w, blk0, nb, kKT, lane);
-                if constexpr (KVT == kKvInt8) {
-                    const uint32_t sd = sbase + kOffScl + s * 256;
-                    copy_int8_scales<BS>(sd, sd + 128, cv, h, w, blk0, nb, lane);
-                }
-                cp_async_mbar_arrive(&bars.code_full[s]);
+                if (j + 1 < ntiles)
+                    w.slide(blk0 + kBPT, lane);
             }
-            if (j + 1 < ntiles)
-                w.slide(blk0 + kBPT, lane);
+            // copies this warp issued land before it exits
+            cp_async_wait_all();
+        } else {
+            // 8-bit codes: each dequant warp loads its own rows one tile
+            // ahead; this warp keeps the lines of up to kPrefetchTiles tiles
+            // past the one being converted on their way into L2, paced by the
+            // count of converted tiles.
+            const volatile int *progress =
+                reinterpret_cast<const volatile int *>(smem + kOffProgress);
+            for (int j = 1; j < ntiles; ++j) {
+                if (j > kPrefetchTiles &&
+                    __shfl_sync(0xffffffffu, *progress, 0) < j - kPrefetchTiles) {
+                    const uint64_t t0 = global_timer_ns();
+                    bool ok = true;
+                    while (__shfl_sync(0xffffffffu, *progress, 0) < j - kPrefetchTiles) {
+                        __nanosleep(128);
+                        // lane 0's clock and status decide, so the warp stays converged
+                        const bool late = __shfl_sync(0xffffffffu,
+                                                      global_timer_ns() - t0 > kWaitLimitNs ||
+                                                          device_wait_failed(p.status),
+                                                      0);
+                        if (late) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!ok)
+                        break;   // the dequant warps stopped: nothing left to prefetch for
+                }
+                w.slide(j * kBPT, lane);
+                prefetch_blocks<BS, KVT>(cv, h, w, j * kBPT, min(kBPT, nblk - j * kBPT), lane);
+            }
         }
-        // copies this warp issued land before it exits
-        cp_async_wait_all();
     } else if (warp == kWarpMma) {
         // --------------------------------------------------- MMA issuer --
-        // S(k) overwrites P(k-2) in the same buffer, so Q K(k)^T is issued
-        // once K(k) is dequantised and P(k-2) V has been issued (the tensor
-        // core executes one thread's MMAs in issue order).  Nothing blocks on
-        // one event while another could proceed; when a round issued
-        // nothing, the warp sleeps (bounded) on the P that is due.
+        // S(k) overwrites P(k - kSBufs) in the same buffer, so Q K(k)^T is
+        // issued once K(k) is dequantised and P(k - kSBufs) V has been issued
+        // (the tensor core executes one thread's MMAs in issue order).  Both
+        // events are polled without blocking: a warp suspended on P(j) would
+        // not issue Q K(j+1)^T the moment K(j+1) is ready, and the softmax
+        // would then wait for S(j+1).  A round that issued nothing sleeps a
+        // few tens of nanoseconds.
         if (ntiles > 0) {
             bool ok = warp_wait(bars.q_full, 0, p.status);
             tc_fence_after();
             const uint64_t kd0 = desc_sw128(sbase + kOffKV, 16, 1024);
             const uint64_t vd0 = desc_sw128(sbase + kOffKV + 16384, 8192, 1024);
-            constexpr uint32_t kPollSleepNs = 200;
+            constexpr uint32_t kPollSleepNs = 20;
             int nqk = 0, nxt = 0;
             uint64_t t_last = 0;
             uint32_t idle = 0;
             while (ok && nxt < ntiles) {
                 bool progressed = false;
-                if (nqk < ntiles && nqk <= nxt + 1 &&
+                if (nqk < ntiles && nqk < nxt + kSBufs &&
                     __any_sync(0xffffffffu, mbar_test_wait(&bars.kv_full[nqk % kKVBufs],
                                                            (nqk / kKVBufs) & 1))) {
                     tc_fence_after();
-                    const uint32_t sd = tmem + kTmS + (nqk & 1) * kKT;
+                    const uint32_t sd = tmem + kTmS + sbuf(nqk) * kKT;
                     const uint64_t kd = kd0 + (uint64_t)(((nqk % kKVBufs) * kKVBuf) >> 4);
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
                         mma_f16_ts_elect(sd, tmem + kTmQ + ks * 8,
                                          kd + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4),
                                          kIdescQK, ks > 0 ? 1u : 0u);
-                    mma_commit_elect(&bars.s_full[nqk & 1]);
+                    mma_commit_elect(&bars.s_full[sbuf(nqk)]);
                     ++nqk;
                     progressed = true;
                 }
                 if (nxt < nqk) {
-                    uint64_t *bar = &bars.p_full[nxt & 1];
-                    const uint32_t par = (nxt >> 1) & 1;
-                    const bool rdy = progressed ? mbar_test_wait(bar, par)
-                                                : mbar_try_wait_for(bar, par, kPollSleepNs);
+                    uint64_t *bar = &bars.p_full[sbuf(nxt)];
+                    const uint32_t par = sphase(nxt);
+                    const bool rdy = mbar_test_wait(bar, par);
                     if (__any_sync(0xffffffffu, rdy)) {
                         tc_fence_after();
-                        const uint32_t pa = tmem + kTmS + (nxt & 1) * kKT;
+                        const uint32_t pa = tmem + kTmS + sbuf(nxt) * kKT;
                         const uint64_t vd = vd0 + (uint64_t)(((nxt % kKVBufs) * kKVBuf) >> 4);
 #pragma unroll
                         for (int ks = 0; ks < kKT / 16; ++ks)
                             mma_f16_ts_elect(tmem + kTmO, pa + ks * 8,
                                              vd + (uint64_t)((ks * 2048) >> 4), kIdescPV,
                                              (nxt > 0 || ks > 0) ? 1u : 0u);
-                        mma_commit_elect(&bars.pv_done[nxt & 1]);
+                        mma_commit_elect(&bars.pv_done[sbuf(nxt)]);
                         mma_commit_elect(&bars.kv_empty[nxt % kKVBufs]);
                         ++nxt;
                         progressed = true;
@@ -308,7 +337,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 }
                 if (progressed) {
                     idle = 0;
-                } else if ((++idle & 15u) == 0) {
+                } else if ((++idle & 15u) != 0) {
+                    __nanosleep(kPollSleepNs);
+                } else {
                     // lane 0's clock decides, so that the warp stays converged
                     const uint64_t now = __shfl_sync(0xffffffffu, global_timer_ns(), 0);
                     if (idle == 16u) {
@@ -323,119 +354,168 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             mma_commit_elect(bars.mma_done);
             warp_wait(bars.mma_done, 0, p.status);
         }
-    } else if (is_dequant_warp(warp)) {
+    } else if (warp < kDequantWarps) {
         // ------------------------------------------------------ dequant --
-        const int row = (warp & 1) * 32 + lane;   // key row of this thread
-        const int isv = (warp == 2 || warp == 3) ? 1 : 0;   // 0: K (warps 0, 1, 6, 7), 1: V
-        const int c0 = warp >= 6 ? 4 : 0;         // first 16-byte chunk of the row
-        const int nch = isv ? 8 : 4;              // chunks this warp converts
-        const float kfac = p.scale_log2;
+        // warps 0-3 convert K, warps 4-7 V; warp w takes key rows
+        // 32 (w & 1) .. +31 of every tile and d half (w >> 1) & 1, one key row
+        // per thread.  Each SM sub-partition (warp % 4) runs one K and one V warp.
+        const int isv = warp >> 2;
+        const int row = (warp & 1) * 32 + lane;   // key row of this thread in a tile
+        const int dh = (warp >> 1) & 1;           // d half: 16-byte code chunks 4 dh .. 4 dh + 3
         if constexpr (KVT == kKvFp16) {
-            // clear the rows no key of this split may read, then release
+            // the copies landed: clear the rows no key of this split may read
+            // (never-written slots may hold NaN patterns, and 0 * NaN in P V
+            // would poison O), then release the buffer to the MMA warp
             for (int j = 0; j < ntiles; ++j) {
                 const int bj = j % kKVBufs;
                 if (!warp_wait(&bars.kv_tma[bj], (j / kKVBufs) & 1, p.status))
                     break;
                 const int key = key_begin + j * kKT + row;
                 if (key >= ctx || j * kKT + row >= nblk * BS) {
-                    // the whole 128-byte row of each d half this warp owns
-                    // (K: half c0 / 4; V: both)
-                    uint8_t *kv = smem + kOffKV + bj * kKVBuf + isv * 16384;
+                    uint8_t *kv = smem + kOffKV + bj * kKVBuf + isv * 16384 + dh * 8192;
                     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        if (!isv && hh != (c0 >> 2))
-                            continue;
-#pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            *reinterpret_cast<uint4 *>(kv + hh * 8192 + row * 128 + c * 16) = z;
-                    }
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4 *>(kv + row * 128 + c * 16) = z;
                 }
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&bars.kv_full[bj]);
             }
-        }
-        for (int j = 0; KVT != kKvFp16 && j < ntiles; ++j) {
-            const int s = j % kCodeStages, bj = j % kKVBufs;
-            if (!warp_wait(&bars.code_full[s], (j / kCodeStages) & 1, p.status))
-                break;
-            if (j >= kKVBufs &&
-                !warp_wait(&bars.kv_empty[bj], ((j - kKVBufs) / kKVBufs) & 1, p.status))
-                break;
-            const uint8_t *codes = smem + kOffCodes + s * kCodeStage + isv * 8192;
-            const uint16_t *scl = reinterpret_cast<const uint16_t *>(smem + kOffScl + s * 256);
-            uint8_t *kv = smem + kOffKV + bj * kKVBuf + isv * 16384;
-            const int key = key_begin + j * kKT + row;
-            const bool live = key < ctx && j * kKT + row < nblk * BS;
-            uint32_t s2 = 0u;
-            if constexpr (KVT == kKvInt8) {
-                const uint32_t sc = scl[64 + row];   // V scale of this key
-                s2 = sc | (sc << 16);
-            }
-            // all eight 16-byte code chunks of the row are loaded before any is
-            // converted: one shared-memory round trip per tile, not eight
-            uint4 wv[8];
+        } else {
+            // Each thread copies its own 64 code bytes of every tile (and the
+            // INT8 scales of its warp's rows, two per even lane) into the code
+            // ring kCodeStages - 1 tiles ahead with 16-byte cp.async, and reads
+            // back only what its warp copied: per-thread copy groups, no
+            // cross-warp handshake.
+            const uint8_t *cache = isv ? p.v_cache : p.k_cache;
+            const uint16_t *scl = isv ? p.v_scale_tok : p.k_scale_tok;
+            const bool want_scale = KVT == kKvInt8 && (isv || dh == 0);
+            const int32_t *bt_row = p.block_table + (size_t)b * p.max_blocks_per_seq + blk_begin;
+            // table entries read stay below this count (past it: block 0)
+            const int nread = min(nblk, p.max_blocks_per_seq - blk_begin);
+            const float kfac = p.scale_log2;
+            auto block_of = [&](int t) {   // physical block of this thread's row of tile t
+                const int e = (t * kKT + row) / BS;
+                int phys = (t < ntiles && e < nread) ? __ldg(bt_row + e) : 0;
+#ifdef PKVQ_BOUNDS_CHECK
+                if (phys < 0 || phys >= p.num_blocks) {
+                    atomicOr(p.status, kStatusBadBlock);
+                    phys = 0;
+                }
+#endif
+                return phys;
+            };
+            // copies of tile t into stage t % kCodeStages (an empty group past the end)
+            auto issue = [&](int t, int phys) {
+                if (t < ntiles) {
+                    const int st = t % kCodeStages;
+                    const size_t y =
+                        ((size_t)phys * p.num_kv_heads + h) * BS + (t * kKT + row) % BS;
+                    const uint8_t *src = cache + y * 128 + 64 * dh;
+                    const uint32_t dst = sbase + kOffCodes + st * kCodeStage + isv * 8192;
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (i < nch)
-                    wv[i] = *reinterpret_cast<const uint4 *>(codes + swz(row, c0 + i));
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if (i >= nch)
+                    for (int i = 0; i < 4; ++i)
+                        cp_async_16(dst + swz(row, 4 * dh + i), src + 16 * i);
+                    if (want_scale && (lane & 1) == 0)   // this row's scale and the next one's
+                        cp_async_4(sbase + kOffScl + (st * kDequantWarps + warp) * 64 + 2 * lane,
+                                   scl + y);
+                }
+                cp_async_commit();
+            };
+            for (int t = 0; t < kCodeStages - 1; ++t)
+                issue(t, block_of(t));
+            int phys_next = block_of(kCodeStages - 1);
+            for (int j = 0; j < ntiles; ++j) {
+                // the stage of tile j - 1 takes tile j + kCodeStages - 1
+                issue(j + kCodeStages - 1, phys_next);
+                phys_next = block_of(j + kCodeStages);   // used by the next round
+                cp_async_wait_group<kCodeStages - 1>();   // this thread's copies of tile j
+                __syncwarp();                             // and the neighbour lanes' scales
+                const int st = j % kCodeStages, bj = j % kKVBufs;
+                if (j >= kKVBufs &&
+                    !warp_wait(&bars.kv_empty[bj], ((j - kKVBufs) / kKVBufs) & 1, p.status))
                     break;
-                const int cc = c0 + i;   // 16-byte code chunk
-                const uint4 w = wv[i];
-                uint32_t hv[8];
-                cvt4<KVT>(w.x, hv[0], hv[1]);
-                cvt4<KVT>(w.y, hv[2], hv[3]);
-                cvt4<KVT>(w.z, hv[4], hv[5]);
-                cvt4<KVT>(w.w, hv[6], hv[7]);
-                if constexpr (KVT == kKvInt8) {
-                    if (isv) {
+                const uint8_t *codes = smem + kOffCodes + st * kCodeStage + isv * 8192;
+                uint4 cur[4];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            __half2 x = __hmul2(*reinterpret_cast<__half2 *>(&hv[e]),
-                                                *reinterpret_cast<const __half2 *>(&s2));
-                            hv[e] = *reinterpret_cast<uint32_t *>(&x);
+                for (int i = 0; i < 4; ++i)
+                    cur[i] = *reinterpret_cast<const uint4 *>(codes + swz(row, 4 * dh + i));
+                uint32_t sc = 0;
+                if (want_scale)
+                    sc = reinterpret_cast<const uint16_t *>(
+                        smem + kOffScl + (st * kDequantWarps + warp) * 64)[lane];
+                uint8_t *kv = smem + kOffKV + bj * kKVBuf + isv * 16384 + dh * 8192;
+                const int key = key_begin + j * kKT + row;
+                const bool live = key < ctx && j * kKT + row < nblk * BS;
+                const uint32_t s2 = sc | (sc << 16);   // INT8 V: the key's scale twice
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    uint32_t hv[8];
+                    cvt4<KVT>(cur[i].x, hv[0], hv[1]);
+                    cvt4<KVT>(cur[i].y, hv[2], hv[3]);
+                    cvt4<KVT>(cur[i].z, hv[4], hv[5]);
+                    cvt4<KVT>(cur[i].w, hv[6], hv[7]);
+                    if constexpr (KVT == kKvInt8) {
+                        if (isv) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                __half2 x = __hmul2(*reinterpret_cast<__half2 *>(&hv[e]),
+                                                    *reinterpret_cast<const __half2 *>(&s2));
+                                hv[e] = *reinterpret_cast<uint32_t *>(&x);
+                            }
                         }
                     }
-                }
-                if (!live) {   // past the context or the split: codes may be anything
+                    if (!live) {   // past the context or the split: codes may be anything
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        hv[e] = 0u;
+                        for (int e = 0; e < 8; ++e)
+                            hv[e] = 0u;
+                    }
+                    // 16 codes -> 32 bytes: chunks 2 i and 2 i + 1 of the row's 128-byte half
+                    *reinterpret_cast<uint4 *>(kv + swz(row, 2 * i)) =
+                        make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                    *reinterpret_cast<uint4 *>(kv + swz(row, 2 * i + 1)) =
+                        make_uint4(hv[4], hv[5], hv[6], hv[7]);
                 }
-                uint8_t *dst = kv + (cc >> 2) * 8192;
-                *reinterpret_cast<uint4 *>(dst + swz(row, (2 * cc) & 7)) =
-                    make_uint4(hv[0], hv[1], hv[2], hv[3]);
-                *reinterpret_cast<uint4 *>(dst + swz(row, (2 * cc + 1) & 7)) =
-                    make_uint4(hv[4], hv[5], hv[6], hv[7]);
-            }
-            if constexpr (KVT == kKvInt8) {
-                if (!isv && c0 == 0) {   // per-key score factor: softmax scale * log2(e) * K scale
-                    float *ksf = reinterpret_cast<float *>(smem + kOffKsf) + bj * 64;
-                    ksf[row] = live ? kfac * __half2float(__ushort_as_half(scl[row])) : 0.0f;
+                if constexpr (KVT == kKvInt8) {
+                    if (!isv && dh == 0) {   // per-key score factor: softmax scale * log2(e) * K scale
+                        float *ksf = reinterpret_cast<float *>(smem + kOffKsf) + bj * 64;
+                        ksf[row] =
+                            live ? kfac * __half2float(__ushort_as_half((uint16_t)sc)) : 0.0f;
+                    }
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&bars.kv_full[bj]);
+                    if (warp == 0)   // prefetch pacing
+                        *reinterpret_cast<volatile int *>(smem + kOffProgress) = j + 1;
                 }
             }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bars.code_empty[s]);
-                mbar_arrive(&bars.kv_full[bj]);
-            }
+            // copies this thread issued land before it exits
+            cp_async_wait_all();
         }
     } else if (warp >= kSoftmaxWarp0) {
         // ------------------------------------------------------ softmax --
-        const int r = tid - 32 * kSoftmaxWarp0;   // row == TMEM lane
         const int sw = warp & 3;           // lane quadrant of this warp
         const uint32_t tl = tmem + ((uint32_t)(32 * sw) << 16);
-        const int tq = r / G, gq = r % G;
-        const bool valid = r < p.rows;
+        // erow: the row in this thread's TMEM lane (Q in, O out); srow: the
+        // row whose scores this thread processes.  Up to 64 rows, row 4 i + q
+        // sits in lane i (< 16) of quadrant q and each lane's two threads
+        // (t, t + 16) take half of its 64 keys each: the exponentials of
+        // padding lanes are not computed.  Otherwise row == lane, one thread
+        // per row.
+        const int erow = kHalf ? (lane < 16 ? 4 * lane + sw : INT_MAX) : 32 * sw + lane;
+        const int srow = kHalf ? 4 * (lane & 15) + sw : erow;
+        const int kh = kHalf ? lane >> 4 : 0;   // key half of this thread
+        constexpr int kCols = kHalf ? kKT / 2 : kKT;   // scores per thread and tile
+        const bool valid = erow < p.rows;
+        const bool svalid = srow < p.rows;
+        const int tq = valid ? erow / G : 0, gq = valid ? erow % G : 0;
         // keys lo..pos are visible to this row (padding rows: the whole split)
-        const int pos = valid ? min(ctx - 1, query_position(p, b, ctx, tq)) : ctx - 1;
-        const int lo = p.window > 0 && valid ? pos - p.window + 1 : INT_MIN;
+        const int pos = svalid ? min(ctx - 1, query_position(p, b, ctx, srow / G)) : ctx - 1;
+        const int lo = p.window > 0 && svalid ? pos - p.window + 1 : INT_MIN;
         // a tile needs masking when it reaches past the lowest position or
         // starts below the highest window start of the rows
         int pos_lo = ctx - 1, lo_hi = INT_MIN;
@@ -473,7 +553,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
         float m_used = -INFINITY, l = 0.0f;
         bool ok = true;
         for (int j = 0; j < ntiles; ++j) {
-            if (!warp_wait(&bars.s_full[j & 1], (j >> 1) & 1, p.status)) {
+            if (!warp_wait(&bars.s_full[sbuf(j)], sphase(j), p.status)) {
                 ok = false;
                 break;
             }
@@ -485,29 +565,36 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 }
             }
             tc_fence_after();
-            float v[kKT];
-            {
+            float v[kCols];
+            if constexpr (kHalf) {
+                uint32_t ua[32];
+                tmem_ld16x2_32(tl + kTmS + sbuf(j) * kKT, ua);
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    v[c] = __uint_as_float(ua[c]);
+            } else {
                 uint32_t ua[32], ub[32];
-                tmem_ld64(tl + kTmS + (j & 1) * kKT, ua, ub);
+                tmem_ld64(tl + kTmS + sbuf(j) * kKT, ua, ub);
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
                     v[c] = __uint_as_float(ua[c]);
                     v[32 + c] = __uint_as_float(ub[c]);
                 }
             }
-            const int key0 = key_begin + j * kKT;
+            const int tile0 = key_begin + j * kKT;   // first key of the tile
+            const int key0 = tile0 + kh * kCols;     // first key of this thread's scores
             if constexpr (KVT != kKvInt8) {
                 const float2 f2 = make_float2(kfac, kfac);
 #pragma unroll
-                for (int c = 0; c < kKT; c += 2) {
+                for (int c = 0; c < kCols; c += 2) {
                     const float2 r2 = __fmul2_rn(make_float2(v[c], v[c + 1]), f2);
                     v[c] = r2.x, v[c + 1] = r2.y;
                 }
             } else {
                 const float *ksf =
-                    reinterpret_cast<const float *>(smem + kOffKsf) + (j % kKVBufs) * 64;
+                    reinterpret_cast<const float *>(smem + kOffKsf) + (j % kKVBufs) * 64 + kh * kCols;
 #pragma unroll
-                for (int c = 0; c < kKT; c += 2) {
+                for (int c = 0; c < kCols; c += 2) {
                     const float2 r2 = __fmul2_rn(make_float2(v[c], v[c + 1]),
                                                  make_float2(ksf[c], ksf[c + 1]));
                     v[c] = r2.x, v[c + 1] = r2.y;
@@ -517,9 +604,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             // split are masked; only tiles that reach past the first row's
             // position or the split's end need it
             const int key_lim = key_begin + nblk * BS;   // first key past the split
-            if (key0 + kKT - 1 > pos_lo || key0 + kKT > key_lim || key0 < lo_hi) {
+            if (tile0 + kKT - 1 > pos_lo || tile0 + kKT > key_lim || tile0 < lo_hi) {
 #pragma unroll
-                for (int c = 0; c < kKT; ++c)
+                for (int c = 0; c < kCols; ++c)
                     if (key0 + c > pos || key0 + c >= key_lim || key0 + c < lo)
                         v[c] = -INFINITY;
             }
@@ -528,29 +615,31 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             for (int i = 0; i < 8; ++i) {
                 m8[i] = v[i];
 #pragma unroll
-                for (int c = i + 8; c < kKT; c += 8)
+                for (int c = i + 8; c < kCols; c += 8)
                     m8[i] = fmaxf(m8[i], v[c]);
             }
-            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            if constexpr (kHalf)   // the row's other key half
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
             // lazy rescale: only when the max grew by more than 2^8
             const bool need = m_used != -INFINITY && mx > m_used + kRescaleLog2;
             if (__any_sync(0xffffffffu, need)) {
                 // O must hold P V of tile j-1 before it is rescaled
-                if (!warp_wait(&bars.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.status)) {
+                if (!warp_wait(&bars.pv_done[sbuf(j - 1)], sphase(j - 1), p.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const float corr = need ? fast_exp2(m_used - mx) : 1.0f;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t o[32];
-                    tmem_ld32(tl + kTmO + 32 * q, o);
+                for (int q = 0; q < 8; ++q) {   // 16 columns at a time: the scores stay live
+                    uint32_t o[16];
+                    tmem_ld16(tl + kTmO + 16 * q, o);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
+                    for (int c = 0; c < 16; ++c)
                         o[c] = __float_as_uint(__uint_as_float(o[c]) * corr);
-                    tmem_st32(tl + kTmO + 32 * q, o);
+                    tmem_st16(tl + kTmO + 16 * q, o);
                 }
                 if (need) {
                     l *= corr;
@@ -563,30 +652,40 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             const float2 nmu = make_float2(-mu, -mu);
             float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                              make_float2(0.f, 0.f)};
-            uint32_t pk[kKT / 2];
+            // P row over the first 32 columns of its S buffer (A operand of
+            // P V), 32 keys (16 columns) at a time
 #pragma unroll
-            for (int c = 0; c < kKT; c += 2) {
-                const float2 d = __fadd2_rn(make_float2(v[c], v[c + 1]), nmu);
-                const float2 e = make_float2(fast_exp2(d.x), fast_exp2(d.y));
-                acc[(c >> 1) & 3] = __fadd2_rn(acc[(c >> 1) & 3], e);
-                pk[c / 2] = pack_half2(e.x, e.y);
+            for (int g = 0; g < kCols / 32; ++g) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    const int cc = 32 * g + c;
+                    const float2 d = __fadd2_rn(make_float2(v[cc], v[cc + 1]), nmu);
+                    const float2 e = make_float2(fast_exp2(d.x), fast_exp2(d.y));
+                    acc[(c >> 1) & 3] = __fadd2_rn(acc[(c >> 1) & 3], e);
+                    pk[c / 2] = pack_half2(e.x, e.y);
+                }
+                if constexpr (kHalf)
+                    tmem_st16x2_16(tl + kTmS + sbuf(j) * kKT, pk);
+                else
+                    tmem_st16(tl + kTmS + sbuf(j) * kKT + 16 * g, pk);
             }
             const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
             const float2 a = __fadd2_rn(a01, a23);
             l += a.x + a.y;
-            // P row over the first 32 columns of its S buffer (A operand of P V)
-            tmem_st32(tl + kTmS + (j & 1) * kKT, pk);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&bars.p_full[j & 1]);
+                mbar_arrive(&bars.p_full[sbuf(j)]);
         }
 
         // ---- epilogue ----
+        if constexpr (kHalf)   // each thread summed its own key half
+            l += __shfl_xor_sync(0xffffffffu, l, 16);
         const int jl = ntiles - 1;   // P V of the last tile retires after all others
         const bool have_o =
-            ok && ntiles > 0 && warp_wait(&bars.pv_done[jl & 1], (jl >> 1) & 1, p.status);
+            ok && ntiles > 0 && warp_wait(&bars.pv_done[sbuf(jl)], sphase(jl), p.status);
         if (have_o)
             tc_fence_after();
         if (si.nsplit == 1) {
@@ -620,7 +719,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 p.lse[qrow] = (have_o && l > 0.0f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
         } else {
             // FP32 partial: unnormalised O, max (log2 units) and sum of row r
-            const size_t wrow = ((size_t)h * p.num_splits + slot) * p.rows_per_cta + r;
+            const size_t wrow = ((size_t)h * p.num_splits + slot) * p.rows_per_cta + erow;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t o[32];
@@ -654,7 +753,7 @@ template <int KVT, int BS>
 cudaError_t launch_tc(const DecodeParams &p, const CUtensorMap &kmap, const CUtensorMap &vmap,
                       cudaStream_t stream)
 {
-    auto kern = decode_tc_kernel<KVT, BS>;
+    auto kern = p.rows <= 64 ? decode_tc_kernel<KVT, BS, true> : decode_tc_kernel<KVT, BS, false>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc);
     if (e != cudaSuccess)

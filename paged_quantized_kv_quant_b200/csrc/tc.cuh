@@ -226,6 +226,30 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *r)
                  : "memory");
 }
 
+// 16-lane shapes (16x32bx2): threads 0-15 access lanes 0-15 of the warp's
+// quadrant (plus the lane offset in taddr) at the given columns, threads
+// 16-31 the same lanes at the columns plus the half-split offset.  Here the
+// split offset equals the repeat count, so a lane's two threads cover 2N
+// consecutive columns: thread t holds lane t % 16, columns N * (t / 16) + 0..N-1.
+__device__ __forceinline__ void tmem_ld16x2_32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x32.b32 " PKVQ_LIST32 ", [%32], 32;\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : PKVQ_R32(r)
+                 : "r"(taddr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16x2_16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile("tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 16, "
+                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                 "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+                 "r"(r[13]), "r"(r[14]), "r"(r[15])
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait()
 {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");

@@ -38,7 +38,8 @@ CASES = [
     (INT8, 8, 1, [2000, 77], 4, 64),        # 32 rows
     (INT8, 16, 2, [3000, 129], 6, 16),      # 48 rows
     (FP8, 32, 4, [2500, 1], 7, 32),         # 56 rows
-    (INT8, 16, 2, [1300, 700], 8, 16),      # 64 rows
+    (INT8, 16, 2, [1300, 700], 8, 16),      # 64 rows: the last half-lane layout
+    (INT8, 16, 2, [1500, 90], 9, 16),       # 72 rows: one thread per row
     (FP8, 16, 2, [900], 16, 16),            # 128 rows: one full tile
     (FP8, 32, 2, [500], 16, 16),            # 256 rows: past the tile, mma.sync row groups
 ]
@@ -207,6 +208,7 @@ WINDOW_CASES = [
     (INT8, 16, 4, [2000, 65], 3, 32, 129),             # 12 rows, window of one row + 1
     (INT8, 32, 4, [5000, 64, 3], 5, 16, 1000),         # tcgen05, 40 rows
     (synth.FP16, 16, 2, [3000], 4, 64, 200),           # tcgen05, FP16
+    (FP8, 16, 2, [2000, 300], 10, 16, 150),            # tcgen05, 80 rows
     (synth.FP8_E5M2, 8, 2, [999], 2, 16, 1),           # window 1: each row its own key
 ]
 
