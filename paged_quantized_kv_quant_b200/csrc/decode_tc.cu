@@ -357,11 +357,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
     } else if (warp < kDequantWarps) {
         // ------------------------------------------------------ dequant --
         // warps 0-3 convert K, warps 4-7 V; warp w takes key rows
-        // 32 (w & 1) .. +31 of every tile and d half (w >> 1) & 1, one key row
-        // per thread.  Each SM sub-partition (warp % 4) runs one K and one V warp.
+        // 16 (w & 3) .. +15 of every tile, thread l row 16 (w & 3) + l % 16 and
+        // d half l / 16 (so 8 consecutive lanes touch 8 consecutive rows of one
+        // half: no bank conflicts).  Each SM sub-partition (warp % 4) runs one
+        // K and one V warp.
         const int isv = warp >> 2;
-        const int row = (warp & 1) * 32 + lane;   // key row of this thread in a tile
-        const int dh = (warp >> 1) & 1;           // d half: 16-byte code chunks 4 dh .. 4 dh + 3
+        const int row0 = 16 * (warp & 3);         // first key row of this warp in a tile
+        const int row = row0 + (lane & 15);       // key row of this thread
+        const int dh = lane >> 4;                 // d half: 16-byte code chunks 4 dh .. 4 dh + 3
         if constexpr (KVT == kKvFp16) {
             // the copies landed: clear the rows no key of this split may read
             // (never-written slots may hold NaN patterns, and 0 * NaN in P V
@@ -384,20 +387,21 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                     mbar_arrive(&bars.kv_full[bj]);
             }
         } else {
-            // Each thread copies its own 64 code bytes of every tile (and the
-            // INT8 scales of its warp's rows, two per even lane) into the code
-            // ring kCodeStages - 1 tiles ahead with 16-byte cp.async, and reads
-            // back only what its warp copied: per-thread copy groups, no
-            // cross-warp handshake.
+            // Each warp copies its own 16 rows of every tile (2 KB: 4 rows x
+            // 128 bytes per instruction, 8 lanes per row, so each instruction
+            // touches 4 cache lines; and the INT8 scales of those rows, 32
+            // bytes) into the code ring kCodeStages - 1 tiles ahead with
+            // 16-byte cp.async, and reads back only what it copied: per-thread
+            // copy groups and a warp barrier, no cross-warp handshake.
             const uint8_t *cache = isv ? p.v_cache : p.k_cache;
             const uint16_t *scl = isv ? p.v_scale_tok : p.k_scale_tok;
-            const bool want_scale = KVT == kKvInt8 && (isv || dh == 0);
             const int32_t *bt_row = p.block_table + (size_t)b * p.max_blocks_per_seq + blk_begin;
             // table entries read stay below this count (past it: block 0)
             const int nread = min(nblk, p.max_blocks_per_seq - blk_begin);
             const float kfac = p.scale_log2;
-            auto block_of = [&](int t) {   // physical block of this thread's row of tile t
-                const int e = (t * kKT + row) / BS;
+            // physical block of this warp's 16 rows of tile t (one block: BS >= 16)
+            auto block_of = [&](int t) {
+                const int e = (t * kKT + row0) / BS;
                 int phys = (t < ntiles && e < nread) ? __ldg(bt_row + e) : 0;
 #ifdef PKVQ_BOUNDS_CHECK
                 if (phys < 0 || phys >= p.num_blocks) {
@@ -411,16 +415,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             auto issue = [&](int t, int phys) {
                 if (t < ntiles) {
                     const int st = t % kCodeStages;
-                    const size_t y =
-                        ((size_t)phys * p.num_kv_heads + h) * BS + (t * kKT + row) % BS;
-                    const uint8_t *src = cache + y * 128 + 64 * dh;
+                    const size_t y0 =
+                        ((size_t)phys * p.num_kv_heads + h) * BS + (t * kKT + row0) % BS;
                     const uint32_t dst = sbase + kOffCodes + st * kCodeStage + isv * 8192;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        cp_async_16(dst + swz(row, 4 * dh + i), src + 16 * i);
-                    if (want_scale && (lane & 1) == 0)   // this row's scale and the next one's
-                        cp_async_4(sbase + kOffScl + (st * kDequantWarps + warp) * 64 + 2 * lane,
-                                   scl + y);
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = 4 * i + (lane >> 3), c = lane & 7;   // row within the warp's 16
+                        cp_async_16(dst + swz(row0 + r, c), cache + (y0 + r) * 128 + 16 * c);
+                    }
+                    if (KVT == kKvInt8 && lane < 2)   // 8 rows' scales per lane
+                        cp_async_16(sbase + kOffScl + (st * kDequantWarps + warp) * 64 + 16 * lane,
+                                    scl + y0 + 8 * lane);
                 }
                 cp_async_commit();
             };
@@ -432,7 +437,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 issue(j + kCodeStages - 1, phys_next);
                 phys_next = block_of(j + kCodeStages);   // used by the next round
                 cp_async_wait_group<kCodeStages - 1>();   // this thread's copies of tile j
-                __syncwarp();                             // and the neighbour lanes' scales
+                __syncwarp();                             // and the other lanes' copies
                 const int st = j % kCodeStages, bj = j % kKVBufs;
                 if (j >= kKVBufs &&
                     !warp_wait(&bars.kv_empty[bj], ((j - kKVBufs) / kKVBufs) & 1, p.status))
@@ -443,9 +448,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                 for (int i = 0; i < 4; ++i)
                     cur[i] = *reinterpret_cast<const uint4 *>(codes + swz(row, 4 * dh + i));
                 uint32_t sc = 0;
-                if (want_scale)
+                if constexpr (KVT == kKvInt8)
                     sc = reinterpret_cast<const uint16_t *>(
-                        smem + kOffScl + (st * kDequantWarps + warp) * 64)[lane];
+                        smem + kOffScl + (st * kDequantWarps + warp) * 64)[lane & 15];
                 uint8_t *kv = smem + kOffKV + bj * kKVBuf + isv * 16384 + dh * 8192;
                 const int key = key_begin + j * kKT + row;
                 const bool live = key < ctx && j * kKT + row < nblk * BS;
