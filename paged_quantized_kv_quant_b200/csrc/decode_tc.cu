@@ -23,12 +23,12 @@
 //   warps 0-7  dequant: code tiles -> fp16 K/V tiles in the 128-byte-
 //              swizzled layout [d half][key][64 d] (the K-major B operand of
 //              Q K^T and the MN-major B operand of P V).  Warps 0-3 convert
-//              K, warps 4-7 V, each one 32-key half of a tile and one d half
-//              (64 codes per thread and tile), so every SM sub-partition runs
-//              one K and one V warp.  Each thread copies its own 64 code bytes
-//              into a 5-stage ring with 16-byte cp.async four tiles ahead and
-//              reads back only those: no producer warp issues the ~1,000
-//              copies of a tile alone, and no barrier hands the codes over.
+//              K, warps 4-7 V, each 16 key rows of a tile (64 codes per thread
+//              and tile), so every SM sub-partition runs one K and one V warp.
+//              Each warp copies its own rows into a 4-stage ring with
+//              coalesced 16-byte cp.async three tiles ahead and reads back
+//              only those: no producer warp issues a tile's copies alone, and
+//              no barrier hands the codes over.
 //   warp 8     TMEM allocation; the whole warp runs the issue loop, one
 //              elected lane issues each tcgen05 instruction.
 //   warp 9     L2 prefetch of the tiles up to kPrefetchTiles ahead of the
@@ -92,7 +92,7 @@ constexpr int kKVBuf = 32768;
 // 8-bit codes: a ring of kCodeStages stages (K 8K, V 8K; rows 128-byte
 // swizzled), each dequant thread copying and reading back only its own bytes;
 // copies run kCodeStages - 1 tiles ahead of the conversion
-constexpr int kCodeStages = 5;
+constexpr int kCodeStages = 4;
 constexpr int kOffCodes = kOffKV + kKVBufs * kKVBuf;
 constexpr int kCodeStage = 16384;
 constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // stages x 8 warps x 32 halves
