@@ -61,7 +61,7 @@
 namespace pkvq {
 namespace {
 
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr int kKT = 64;              // keys per tile
 // 4 K/V buffers: issuing Q K^T two tiles ahead holds tiles j, j+1 and j+2,
 // and the fourth lets the dequantisation of j+3 start before P(j) V has
@@ -77,6 +77,7 @@ constexpr int kDequantWarps = 8;   // warps 0-7
 constexpr int kWarpMma = 8;
 constexpr int kWarpPf = 9;         // L2 prefetch (FP16: the copies)
 constexpr int kSoftmaxWarp0 = 10;  // warps 10-13: lane quadrants 2, 3, 0, 1
+constexpr int kWarpPv = 14;        // issues P V (warp 8 issues Q K^T)
 
 // tensor memory: S/P buffers 0 and 1 (P in the first 32 columns of its
 // buffer), O, Q (two fp16 per column)
@@ -282,74 +283,52 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             }
         }
     } else if (warp == kWarpMma) {
-        // --------------------------------------------------- MMA issuer --
-        // S(k) overwrites P(k - kSBufs) in the same buffer, so Q K(k)^T is
-        // issued once K(k) is dequantised and P(k - kSBufs) V has been issued
-        // (the tensor core executes one thread's MMAs in issue order).  Both
-        // events are polled without blocking: a warp suspended on P(j) would
-        // not issue Q K(j+1)^T the moment K(j+1) is ready, and the softmax
-        // would then wait for S(j+1).  A round that issued nothing sleeps a
-        // few tens of nanoseconds.
+        // ------------------------------------------------ Q K^T issuer --
+        // Two issuing warps, one per product: a thread's tcgen05.mma returns
+        // only once the tensor core has accepted it, so a single issuer that
+        // is queueing Q K(j+2)^T cannot issue P(j+1) V the moment P(j+1) is
+        // ready.  S(k) overwrites P(k - kSBufs) in the same columns: Q K(k)^T
+        // waits for that P V to complete (another thread issued it).
         if (ntiles > 0) {
             bool ok = warp_wait(bars.q_full, 0, p.status);
             tc_fence_after();
             const uint64_t kd0 = desc_sw128(sbase + kOffKV, 16, 1024);
+            for (int k = 0; ok && k < ntiles; ++k) {
+                if (!warp_wait(&bars.kv_full[k % kKVBufs], (k / kKVBufs) & 1, p.status))
+                    break;
+                if (k >= kSBufs &&
+                    !warp_wait(&bars.pv_done[sbuf(k - kSBufs)], sphase(k - kSBufs), p.status))
+                    break;
+                tc_fence_after();
+                const uint32_t sd = tmem + kTmS + sbuf(k) * kKT;
+                const uint64_t kd = kd0 + (uint64_t)(((k % kKVBufs) * kKVBuf) >> 4);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_f16_ts_elect(sd, tmem + kTmQ + ks * 8,
+                                     kd + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4),
+                                     kIdescQK, ks > 0 ? 1u : 0u);
+                mma_commit_elect(&bars.s_full[sbuf(k)]);
+            }
+        }
+    } else if (warp == kWarpPv) {
+        // --------------------------------------------------- P V issuer --
+        // P(j) follows S(j), which followed K(j) and V(j) (one barrier for
+        // both halves of the buffer).  Its last commit covers every product:
+        // each Q K^T completed before the P V of the same tile was issued.
+        if (ntiles > 0) {
             const uint64_t vd0 = desc_sw128(sbase + kOffKV + 16384, 8192, 1024);
-            constexpr uint32_t kPollSleepNs = 20;
-            int nqk = 0, nxt = 0;
-            uint64_t t_last = 0;
-            uint32_t idle = 0;
-            while (ok && nxt < ntiles) {
-                bool progressed = false;
-                if (nqk < ntiles && nqk < nxt + kSBufs &&
-                    __any_sync(0xffffffffu, mbar_test_wait(&bars.kv_full[nqk % kKVBufs],
-                                                           (nqk / kKVBufs) & 1))) {
-                    tc_fence_after();
-                    const uint32_t sd = tmem + kTmS + sbuf(nqk) * kKT;
-                    const uint64_t kd = kd0 + (uint64_t)(((nqk % kKVBufs) * kKVBuf) >> 4);
+            for (int j = 0; j < ntiles; ++j) {
+                if (!warp_wait(&bars.p_full[sbuf(j)], sphase(j), p.status))
+                    break;
+                tc_fence_after();
+                const uint32_t pa = tmem + kTmS + sbuf(j) * kKT;
+                const uint64_t vd = vd0 + (uint64_t)(((j % kKVBufs) * kKVBuf) >> 4);
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_f16_ts_elect(sd, tmem + kTmQ + ks * 8,
-                                         kd + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4),
-                                         kIdescQK, ks > 0 ? 1u : 0u);
-                    mma_commit_elect(&bars.s_full[sbuf(nqk)]);
-                    ++nqk;
-                    progressed = true;
-                }
-                if (nxt < nqk) {
-                    uint64_t *bar = &bars.p_full[sbuf(nxt)];
-                    const uint32_t par = sphase(nxt);
-                    const bool rdy = mbar_test_wait(bar, par);
-                    if (__any_sync(0xffffffffu, rdy)) {
-                        tc_fence_after();
-                        const uint32_t pa = tmem + kTmS + sbuf(nxt) * kKT;
-                        const uint64_t vd = vd0 + (uint64_t)(((nxt % kKVBufs) * kKVBuf) >> 4);
-#pragma unroll
-                        for (int ks = 0; ks < kKT / 16; ++ks)
-                            mma_f16_ts_elect(tmem + kTmO, pa + ks * 8,
-                                             vd + (uint64_t)((ks * 2048) >> 4), kIdescPV,
-                                             (nxt > 0 || ks > 0) ? 1u : 0u);
-                        mma_commit_elect(&bars.pv_done[sbuf(nxt)]);
-                        mma_commit_elect(&bars.kv_empty[nxt % kKVBufs]);
-                        ++nxt;
-                        progressed = true;
-                    }
-                }
-                if (progressed) {
-                    idle = 0;
-                } else if ((++idle & 15u) != 0) {
-                    __nanosleep(kPollSleepNs);
-                } else {
-                    // lane 0's clock decides, so that the warp stays converged
-                    const uint64_t now = __shfl_sync(0xffffffffu, global_timer_ns(), 0);
-                    if (idle == 16u) {
-                        t_last = now;
-                    } else if (now - t_last > kWaitLimitNs) {
-                        if (lane == 0)
-                            atomicOr(p.status, kStatusWaitTimeout);
-                        ok = false;
-                    }
-                }
+                for (int ks = 0; ks < kKT / 16; ++ks)
+                    mma_f16_ts_elect(tmem + kTmO, pa + ks * 8, vd + (uint64_t)((ks * 2048) >> 4),
+                                     kIdescPV, (j > 0 || ks > 0) ? 1u : 0u);
+                mma_commit_elect(&bars.pv_done[sbuf(j)]);
+                mma_commit_elect(&bars.kv_empty[j % kKVBufs]);
             }
             mma_commit_elect(bars.mma_done);
             warp_wait(bars.mma_done, 0, p.status);
