@@ -18,7 +18,7 @@
 // tile, tensor memory holds two S buffers: S(j+2) = Q K(j+2)^T is issued as
 // soon as P(j) V has been, and the softmax finds its next S ready.
 //
-// Warp roles (14 warps; the softmax warps form one aligned group of four, as
+// Warp roles (15 warps; the softmax warps form one aligned group of four, as
 // each warp reaches only the tensor-memory lanes 32 * (warp % 4) + 0..31):
 //   warps 0-7  dequant: code tiles -> fp16 K/V tiles in the 128-byte-
 //              swizzled layout [d half][key][64 d] (the K-major B operand of
@@ -29,8 +29,11 @@
 //              coalesced 16-byte cp.async three tiles ahead and reads back
 //              only those: no producer warp issues a tile's copies alone, and
 //              no barrier hands the codes over.
-//   warp 8     TMEM allocation; the whole warp runs the issue loop, one
-//              elected lane issues each tcgen05 instruction.
+//   warp 8     TMEM allocation and the Q K^T products, warp 14 the P V
+//              products: a thread's tcgen05.mma returns only once the tensor
+//              core has taken it, so one issuer queueing Q K(j+2)^T would
+//              delay P(j+1) V.  One elected lane of the (converged) warp
+//              issues each tcgen05 instruction.
 //   warp 9     L2 prefetch of the tiles up to kPrefetchTiles ahead of the
 //              conversion (FP16 caches: also the copies, see below).
 //   warps 10-13 softmax: Q rows into tensor memory, S read with tcgen05.ld,
