@@ -40,6 +40,8 @@ CASES = [
     (FP8, 32, 4, [2500, 1], 7, 32),         # 56 rows
     (INT8, 16, 2, [1300, 700], 8, 16),      # 64 rows: the last half-lane layout
     (INT8, 16, 2, [1500, 90], 9, 16),       # 72 rows: one thread per row
+    (FP8, 9, 1, [700, 33], 2, 16),          # 18 rows (G = 9): near the fewest on tcgen05
+    (INT8, 20, 2, [1200, 250], 10, 32),     # 100 rows, two threads' worth of lanes idle
     (FP8, 16, 2, [900], 16, 16),            # 128 rows: one full tile
     (FP8, 32, 2, [500], 16, 16),            # 256 rows: past the tile, mma.sync row groups
 ]
