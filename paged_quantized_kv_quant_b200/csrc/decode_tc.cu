@@ -102,7 +102,7 @@ constexpr int kCodeStage = 16384;
 constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // stages x 8 warps x 32 halves
 constexpr int kOffKsf = kOffScl + kCodeStages * kDequantWarps * 64;   // bufs x 64 fp32 K factors
 constexpr int kOffBars = kOffKsf + kKVBufs * 64 * 4;
-constexpr int kNumBars = 1 + 3 * kKVBufs + 3 * kSBufs + 1;
+constexpr int kNumBars = 1 + 3 * kKVBufs + 3 * kSBufs + 2;
 constexpr int kOffTaddr = kOffBars + kNumBars * 8;
 constexpr int kOffProgress = kOffTaddr + 8;   // tiles dequantised so far (prefetch pacing)
 constexpr int kSmemBytes = kOffProgress + 8;
@@ -116,7 +116,7 @@ struct Bars {
     uint64_t *q_full;
     uint64_t *kv_full, *kv_empty;       // [kKVBufs]
     uint64_t *s_full, *p_full, *pv_done;   // [S/P buffer]
-    uint64_t *mma_done;
+    uint64_t *mma_done, *qk_done;      // each issuer's products retired (before TMEM is freed)
     uint64_t *kv_tma;                   // [kKVBufs] FP16: the buffer's copies landed
 };
 
@@ -131,7 +131,8 @@ __device__ __forceinline__ Bars carve_bars(uint8_t *smem)
     r.p_full = r.s_full + kSBufs;
     r.pv_done = r.p_full + kSBufs;
     r.mma_done = r.pv_done + kSBufs;
-    r.kv_tma = r.mma_done + 1;
+    r.qk_done = r.mma_done + 1;
+    r.kv_tma = r.qk_done + 1;
     return r;
 }
 
@@ -190,6 +191,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
             mbar_init(&bars.pv_done[i], 1);
         }
         mbar_init(bars.mma_done, 1);
+        mbar_init(bars.qk_done, 1);
         fence_mbar_init();
     }
     // Inputs may come from the previous kernel: wait for it to complete.
@@ -312,6 +314,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap,
                                      kIdescQK, ks > 0 ? 1u : 0u);
                 mma_commit_elect(&bars.s_full[sbuf(k)]);
             }
+            // all of this thread's products retired before tensor memory is
+            // freed (on an early exit some may still be running)
+            mma_commit_elect(bars.qk_done);
+            warp_wait(bars.qk_done, 0, p.status);
         }
     } else if (warp == kWarpPv) {
         // --------------------------------------------------- P V issuer --
