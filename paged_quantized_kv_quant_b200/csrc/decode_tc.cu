@@ -94,12 +94,12 @@ __device__ __forceinline__ uint32_t sphase(int j) { return (uint32_t)(j / kSBufs
 constexpr int kOffKV = 0;                                 // bufs x (K 8K+8K, V 8K+8K)
 constexpr int kKVBuf = 32768;
 // 8-bit codes: a ring of kCodeStages stages (K 8K, V 8K; rows 128-byte
-// swizzled), each dequant thread copying and reading back only its own bytes;
+// swizzled), each dequant warp copying and reading back only its own 16 rows;
 // copies run kCodeStages - 1 tiles ahead of the conversion
 constexpr int kCodeStages = 4;
 constexpr int kOffCodes = kOffKV + kKVBufs * kKVBuf;
 constexpr int kCodeStage = 16384;
-constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // stages x 8 warps x 32 halves
+constexpr int kOffScl = kOffCodes + kCodeStages * kCodeStage;   // stages x 8 warps x 32 halves (16 used)
 constexpr int kOffKsf = kOffScl + kCodeStages * kDequantWarps * 64;   // bufs x 64 fp32 K factors
 constexpr int kOffBars = kOffKsf + kKVBufs * 64 * 4;
 constexpr int kNumBars = 1 + 3 * kKVBufs + 3 * kSBufs + 2;
