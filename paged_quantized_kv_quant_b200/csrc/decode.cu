@@ -830,7 +830,6 @@ decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
 template <int BS>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
 {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long gw = (long long)blockIdx.x * 4 + warp;
     const long long total = (long long)p.batch * p.num_kv_heads * p.rows;
@@ -844,16 +843,14 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
     MergeRow mr;
     mr.row0 = (size_t)y * p.num_splits * p.rows_per_cta + rr % p.rows_per_cta;
     mr.stride = p.rows_per_cta;
-    // The first chunk is loaded for the slots all sequences at
-    // max_context_len would give, while the real slots are computed from the
-    // context lengths; it is reloaded only when they differ.
-    const int gfirst = b * p.uniform_splits;
-    mr.load(p, gfirst, p.uniform_splits, 0, lane);
+    // The slots of sequence b come from the context lengths, inputs the split
+    // kernel does not write: they are found while the split kernel's last
+    // CTAs still run, and only the partials wait for its completion.
     const SplitInfo si = find_split<BS>(p, -1, b);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (si.nsplit <= 1)
         return;   // a single split wrote the final row itself
-    if (si.first != gfirst || si.nsplit != p.uniform_splits)
-        mr.load(p, si.first, si.nsplit, 0, lane);
+    mr.load(p, si.first, si.nsplit, 0, lane);
     mr.finish(p, si.first, si.nsplit, b, h, rr, lane);
 }
 
